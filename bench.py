@@ -1,0 +1,475 @@
+#!/usr/bin/env python
+"""Benchmark of the MoE layer forward on B200: tokens/s and fraction of roofline.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME] [--impl ours|reference]
+
+One step = one ``moe_layer_forward`` (router -> dispatch -> grouped expert FFN
+-> combine) over one batch of synthetic tokens whose inputs are resident in
+HBM.  The default workload is the Mixtral-shaped layer (T=4096, d=4096, N=8,
+k=2, SwiGLU H=14336, bf16).  For N > 1 (torchrun) every rank runs its own
+replica on its own tokens (weak scaling, no data-path collective); the time is
+the max over ranks and ``value`` counts the tokens of all ranks.
+
+``--impl reference`` times the CPU oracle (fp64, the reference arm) on a
+bounded sample of the same workload on this host's cores.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import synth  # noqa: E402
+
+METRIC = "MoE-layer fwd tokens/s on 1 B200 + % of roofline (HBM GB/s or BF16 TFLOP/s)"
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+
+
+# ----------------------------------------------------------------- helpers
+def peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as f:
+            d = json.load(f)
+        return d, "measured"
+    return dict(FALLBACK_PEAKS), "fallback"
+
+
+def env_rank():
+    return (int(os.environ.get("RANK", "0")), int(os.environ.get("LOCAL_RANK", "0")),
+            int(os.environ.get("WORLD_SIZE", "1")))
+
+
+def mult(wl):
+    return 3 if wl.act == "swiglu" else 2
+
+
+def algorithmic(wl, kept: np.ndarray):
+    """Active FLOPs and algorithmic bytes of one layer forward (touched expert
+    weights + x + y + W_g (+ bias, shared expert)); per-stage FLOPs/bytes of
+    the expert up-projection."""
+    es = 4 if wl.dtype == "f32" else 2
+    m = mult(wl)
+    R = int(kept.sum())
+    touched = int(np.count_nonzero(kept))
+    flops = 2.0 * wl.T * wl.N * wl.d + R * 2.0 * m * wl.d * wl.H
+    wbytes = touched * m * wl.d * wl.H * es
+    if wl.H_shared:
+        flops += wl.T * 2.0 * m * wl.d * wl.H_shared
+        wbytes += m * wl.d * wl.H_shared * es
+    abytes = 2 * wl.T * wl.d * es + wl.N * wl.d * es + (wl.N * 4 if wl.bias_std > 0 else 0)
+    up_mult = 2 if wl.act == "swiglu" else 1
+    up_flops = R * 2.0 * wl.d * wl.H * up_mult
+    up_bytes = touched * up_mult * wl.d * wl.H * es          # weights read
+    up_bytes += R * wl.d * (1 if wl.dispatch == "fp8" else es) + R * wl.H * es  # A rows in, h out
+    return dict(flops=flops, bytes=wbytes + abytes, R=R, touched=touched,
+                up_flops=up_flops, up_bytes=up_bytes)
+
+
+class Clocks:
+    """nvidia-smi sampling of SM clocks and throttle reasons during a region."""
+    FIELDS = ("clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.hw_slowdown,"
+              "clocks_event_reasons.hw_thermal_slowdown,clocks_event_reasons.sw_thermal_slowdown,"
+              "clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, index: int):
+        self.index = index
+        self.proc = None
+
+    def __enter__(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", str(self.index), f"--query-gpu={self.FIELDS}",
+                 "--format=csv,noheader,nounits", "-lms", "200"],
+                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except OSError:
+            self.proc = None
+        return self
+
+    def __exit__(self, *a):
+        self.out = ""
+        if self.proc is not None:
+            self.proc.terminate()
+            try:
+                self.out, _ = self.proc.communicate(timeout=5)
+            except subprocess.TimeoutExpired:
+                self.proc.kill()
+                self.out, _ = self.proc.communicate()
+
+    def summary(self):
+        sm, mx, reasons = [], [], set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for line in (self.out or "").splitlines():
+            f = [x.strip() for x in line.split(",")]
+            if len(f) < 7:
+                continue
+            try:
+                sm.append(float(f[0]))
+                mx.append(float(f[1]))
+            except ValueError:
+                continue
+            for n, v in zip(names, f[3:7]):
+                if v.lower().startswith("active"):
+                    reasons.add(n)
+        if not sm:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": [], "samples": 0}
+        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": max(mx), "reasons": sorted(reasons),
+                "samples": len(sm)}
+
+
+def traffic_from_profile(kernel_key: str, workload_key: str):
+    """DRAM bytes per launch from the committed ncu summary, if it was taken
+    on the current kernel source (else None)."""
+    p = os.path.join(ROOT, "profiles", f"{kernel_key}_{workload_key}.txt")
+    if not os.path.exists(p):
+        return None
+    vals = {}
+    with open(p) as f:
+        for line in f:
+            if ":" in line and not line.startswith("#"):
+                k, v = line.split(":", 1)
+                vals[k.strip()] = v.strip()
+    src = os.path.join(ROOT, "top_routing_expert_warp_b200", "csrc", "gemm_tc.cu")
+    h = hashlib.sha256(open(src, "rb").read()).hexdigest()[:16]
+    if vals.get("source_sha256_16") != h:
+        return None
+    try:
+        return float(vals["dram_bytes_per_launch"])
+    except (KeyError, ValueError):
+        return None
+
+
+# ----------------------------------------------------------------- oracle legs
+def oracle_sample(wl, budget_s: float, max_tokens: int = 64):
+    """Time the CPU oracle on a bounded sample of the workload's tokens.
+
+    Routing (router + dispatch) of the sampled tokens and their expert rows and
+    combine.  Returns (tokens/s, tokens, seconds, description)."""
+    import oracle
+    host = synth.make_host(wl, names={"x", "Wg", "bias", "Ws1", "Ws3", "Ws2"})
+
+    def expert(e):
+        return (synth.expert_slice(wl, "W1", e),
+                synth.expert_slice(wl, "W3", e) if wl.act == "swiglu" else None,
+                synth.expert_slice(wl, "W2", e))
+    cache = {}
+
+    def get_expert(e):
+        if e not in cache:
+            cache[e] = expert(e)
+        return cache[e]
+
+    shared = (host["Ws1"], host.get("Ws3"), host["Ws2"]) if wl.H_shared else None
+
+    def run(tokens):
+        t0 = time.perf_counter()
+        sub = wl.with_(T=len(tokens), capacity_factor=0.0)
+        xs = host["x"][tokens]
+        r = oracle.route(sub, xs, host["Wg"], host.get("bias"))
+        oracle.forward_rows_lazy(sub, xs, r, np.arange(len(tokens)), get_expert, shared)
+        return time.perf_counter() - t0
+
+    # warm the weight cache outside the timed region (weights are resident, like HBM)
+    for e in range(wl.N):
+        get_expert(e)
+    pilot = run(np.arange(1))
+    n = int(max(1, min(max_tokens, budget_s / max(pilot, 1e-3))))
+    toks = np.linspace(0, wl.T - 1, n).astype(np.int64)
+    secs = run(toks)
+    desc = (f"{n} of {wl.T} tokens (router, top-k, dispatch and expert FFN + combine of their "
+            f"{n * wl.k} rows; capacity not applied to the sample), fp64, "
+            f"{len(os.sched_getaffinity(0))} host threads (OpenMP)")
+    return n / secs, n, secs, desc
+
+
+def run_reference(args, wl):
+    rank, _, world = env_rank()
+    if rank != 0:
+        return 0
+    cores = len(os.sched_getaffinity(0))
+    # size each step so the whole run stays within a few minutes
+    per_step_budget = min(2.0, 150.0 / max(1, args.steps + args.warmup))
+    rate0, n0, s0, desc = oracle_sample(wl, per_step_budget, max_tokens=8)
+    times = []
+    for i in range(args.warmup + args.steps):
+        rate, n, s, _ = oracle_sample(wl, per_step_budget, max_tokens=8) if i == 0 else (None, n0, None, None)
+        if i >= args.warmup:
+            t0 = time.perf_counter()
+            _oracle_tokens(wl, n0)
+            times.append(time.perf_counter() - t0)
+    ms = 1000.0 * statistics.mean(times) if times else float("nan")
+    value = n0 / (ms / 1000.0)
+    line = {"impl": "reference", "metric": METRIC, "value": value, "unit": "tokens/s",
+            "n_gpus": world, "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+            "data": "synthetic", "config": config_of(wl),
+            "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": cores, "kind": "oracle",
+                             "sample": f"each step: {desc}"},
+            "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0,
+                    "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+_REF_STATE = {}
+
+
+def _oracle_tokens(wl, n):
+    """One reference step: the oracle forward of n evenly spaced tokens."""
+    import oracle
+    st = _REF_STATE.get(wl.name)
+    if st is None:
+        host = synth.make_host(wl, names={"x", "Wg", "bias", "Ws1", "Ws3", "Ws2"})
+        experts = {e: (synth.expert_slice(wl, "W1", e),
+                       synth.expert_slice(wl, "W3", e) if wl.act == "swiglu" else None,
+                       synth.expert_slice(wl, "W2", e)) for e in range(wl.N)}
+        st = _REF_STATE[wl.name] = (host, experts)
+    host, experts = st
+    toks = np.linspace(0, wl.T - 1, n).astype(np.int64)
+    sub = wl.with_(T=n, capacity_factor=0.0)
+    xs = host["x"][toks]
+    r = oracle.route(sub, xs, host["Wg"], host.get("bias"))
+    shared = (host["Ws1"], host.get("Ws3"), host["Ws2"]) if wl.H_shared else None
+    oracle.forward_rows_lazy(sub, xs, r, np.arange(n), lambda e: experts[e], shared)
+
+
+def config_of(wl):
+    c = {"workload": wl.name, "T": wl.T, "d": wl.d, "N": wl.N, "k": wl.k, "H": wl.H,
+         "act": wl.act, "gate_mode": wl.gate_mode, "renormalize": wl.renormalize,
+         "capacity_factor": wl.capacity_factor, "H_shared": wl.H_shared,
+         "dispatch": wl.dispatch_dtype, "seed": wl.seed,
+         "l2": "inputs larger than L2: expert weights read every step exceed 126 MB and the "
+               "token batch rotates over 4 resident copies"}
+    return c
+
+
+# ----------------------------------------------------------------- our arm
+def run_ours(args, wl):
+    import torch
+    import top_routing_expert_warp_b200 as moe
+
+    rank, local, world = env_rank()
+    torch.cuda.set_device(local)
+    dist = None
+    if world > 1:
+        import datetime
+        import torch.distributed as dist
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
+
+    def barrier():
+        if dist is not None:
+            dist.barrier()
+
+    dev = {}
+    t_up = time.perf_counter()
+    for name, shape, std, dt in synth.tensor_specs(wl):
+        tdt = torch.float32 if dt == "f32" else torch.bfloat16
+        t = torch.empty(shape, dtype=tdt, device="cuda")
+        n = int(np.prod(shape))
+        per = int(np.prod(shape[1:])) if len(shape) == 3 else n
+        pinned = torch.empty(per, dtype=tdt, pin_memory=True)
+        pin_np = pinned.view(torch.int16 if dt == "bf16" else torch.float32).numpy()
+        flat = t.view(-1)
+        for s0 in range(0, n, per):
+            synth.normal(wl.seed, synth.TENSOR_IDS[name], per, std, dt, start=s0,
+                         out=pin_np.view(np.uint16) if dt == "bf16" else pin_np)
+            flat[s0:s0 + per].copy_(pinned)
+        dev[name] = t
+    gen_s = time.perf_counter() - t_up
+    cfg = moe.make_config(wl.T, wl.d, wl.N, wl.k, wl.H, H_shared=wl.H_shared,
+                          capacity_factor=wl.capacity_factor, gate_mode=wl.gate_mode,
+                          renormalize=wl.renormalize, act=wl.act, dtype=wl.dtype,
+                          dispatch_dtype=wl.dispatch or None, aux_alpha=wl.aux_alpha)
+    ws = moe.workspace(cfg)
+    tdt = dev["x"].dtype
+    # 4 resident token batches (distinct seeds), rotated per step
+    xs = [dev["x"]]
+    for i in range(1, 4):
+        x = torch.empty_like(dev["x"])
+        x.view(-1).copy_(torch.from_numpy(
+            synth.normal(wl.seed + 1000 * i, 0, wl.T * wl.d, 1.0, wl.dtype).view(
+                np.int16 if wl.dtype == "bf16" else np.float32)).view(tdt).to("cuda"))
+        xs.append(x)
+    y = torch.empty((wl.T, wl.d), dtype=tdt, device="cuda")
+    idx = torch.empty((wl.T, wl.k), dtype=torch.int32, device="cuda")
+    gw = torch.empty((wl.T, wl.k), dtype=torch.float32, device="cuda")
+    counts = torch.empty(wl.N, dtype=torch.int32, device="cuda")
+    f = torch.empty(wl.N, dtype=torch.float32, device="cuda")
+    pm = torch.empty(wl.N, dtype=torch.float32, device="cuda")
+    aux = torch.empty(1, dtype=torch.float32, device="cuda")
+    stream = torch.cuda.current_stream()
+
+    def step(i, x=None):
+        moe.moe_layer_forward(cfg, xs[i % 4] if x is None else x, dev["Wg"], dev.get("bias"),
+                              dev["W1"], dev.get("W3"), dev["W2"], dev.get("Ws1"), dev.get("Ws3"),
+                              dev.get("Ws2"), y, idx, gw, counts, f, pm, aux, ws, stream)
+
+    for i in range(args.warmup):
+        step(i)
+    torch.cuda.synchronize()
+    st, word = moe.moe_check_status(ws)
+    if st != moe.MOE_OK:
+        raise RuntimeError(f"device status after warm-up: {moe.status_string(st)} ({word:#x})")
+    kept_steps = []
+    for i in range(4):                       # routing of each rotated batch
+        step(i)
+        torch.cuda.synchronize()
+        kept = counts.cpu().numpy().astype(np.int64)
+        if wl.capacity_factor > 0:
+            kept = np.minimum(kept, wl.capacity())
+        kept_steps.append(kept)
+
+    # ---- timed region (device events, max over ranks)
+    barrier()
+    torch.cuda.synchronize()
+    l0 = moe.moe_launch_count()
+    moe.moe_profile_begin(args.steps)
+    e0 = torch.cuda.Event(enable_timing=True)
+    e1 = torch.cuda.Event(enable_timing=True)
+    with Clocks(local) as clk:
+        e0.record(stream)
+        for i in range(args.steps):
+            step(i)
+        e1.record(stream)
+        torch.cuda.synchronize()
+    stages, nrec = moe.moe_profile_end()
+    launches = moe.moe_launch_count() - l0
+    barrier()
+    ms_total = e0.elapsed_time(e1)
+    if dist is not None:
+        t = torch.tensor([ms_total], device="cuda")
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        ms_total = float(t.item())
+    ms = ms_total / args.steps
+    st, word = moe.moe_check_status(ws)
+    if st != moe.MOE_OK:
+        raise RuntimeError(f"device status after timing: {moe.status_string(st)} ({word:#x})")
+
+    # ---- end to end through the C ABI with host buffers (pinned)
+    x_host = [xs[i].cpu().pin_memory() for i in range(4)]
+    y_host = torch.empty((wl.T, wl.d), dtype=tdt).pin_memory()
+    xin = torch.empty_like(xs[0])
+    e_steps = max(3, min(args.steps, 50))
+    barrier()
+    torch.cuda.synchronize()
+    a0 = torch.cuda.Event(enable_timing=True)
+    a1 = torch.cuda.Event(enable_timing=True)
+    a0.record(stream)
+    for i in range(e_steps):
+        xin.copy_(x_host[i % 4], non_blocking=True)
+        step(i, xin)
+        y_host.copy_(y, non_blocking=True)
+    a1.record(stream)
+    torch.cuda.synchronize()
+    barrier()
+    e2e_ms = a0.elapsed_time(a1)
+    if dist is not None:
+        t = torch.tensor([e2e_ms], device="cuda")
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        e2e_ms = float(t.item())
+    e2e_ms /= e_steps
+
+    pk, pk_src = peaks()
+    out = None
+    if rank == 0:
+        alg = [algorithmic(wl, k) for k in kept_steps]
+        flops = statistics.mean(a["flops"] for a in alg)
+        byts = statistics.mean(a["bytes"] for a in alg)
+        up_flops = statistics.mean(a["up_flops"] for a in alg)
+        up_bytes = statistics.mean(a["up_bytes"] for a in alg)
+        peak_tf_s = pk["bf16_tflops_sustained"]
+        peak_tf_b = pk["bf16_tflops"]
+        peak_bw = pk["hbm_gbs"]
+        up_ms = stages["expert_up"] / max(1, nrec)
+        # bound of the dominant kernel: arithmetic intensity vs the ridge point
+        ridge = peak_tf_s * 1e12 / (peak_bw * 1e9)
+        tensor_bound = (up_flops / max(up_bytes, 1)) >= ridge
+        if tensor_bound:
+            achieved = up_flops / (up_ms * 1e-3) / 1e12
+            roof = {"kernel": "grouped_gemm_tc (expert up-projection + SwiGLU/ReLU epilogue)",
+                    "bound": "tensor", "achieved": achieved, "peak": peak_tf_s, "unit": "TFLOP/s",
+                    "frac": achieved / peak_tf_s, "peak_kind": f"bf16_tflops_sustained ({pk_src})",
+                    "frac_of_burst_peak": achieved / peak_tf_b,
+                    "algorithmic_per_launch": up_flops, "launch_ms": up_ms}
+        else:
+            achieved = up_bytes / (up_ms * 1e-3) / 1e9
+            roof = {"kernel": "grouped_gemm_tc (expert up-projection + SwiGLU/ReLU epilogue)",
+                    "bound": "hbm", "achieved": achieved, "peak": peak_bw, "unit": "GB/s",
+                    "frac": achieved / peak_bw, "peak_kind": f"hbm_gbs ({pk_src})",
+                    "algorithmic_per_launch": up_bytes, "launch_ms": up_ms}
+        roof["traffic"] = traffic_from_profile("grouped_gemm_up", wl_key(wl))
+        # the whole layer against its own roofline (slower of the two bounds)
+        t_roof_meas = max(flops / (peak_tf_b * 1e12), byts / (peak_bw * 1e9))
+        t_roof_spec = max(flops / 2.25e15, byts / 8.0e12)
+        layer = {"active_flops": flops, "algorithmic_bytes": byts,
+                 "bound": "tensor" if flops / (peak_tf_b * 1e12) >= byts / (peak_bw * 1e9) else "hbm",
+                 "roofline_ms_measured_peaks": 1e3 * t_roof_meas,
+                 "roofline_ms_spec_peaks": 1e3 * t_roof_spec,
+                 "frac_of_roofline_measured": 1e3 * t_roof_meas / ms,
+                 "frac_of_roofline_spec": 1e3 * t_roof_spec / ms}
+        cpu = None
+        if world == 1 and not args.no_cpu_baseline:
+            rate, n, secs, desc = oracle_sample(wl, args.cpu_budget)
+            cpu = {"value": rate, "unit": "tokens/s", "cores": len(os.sched_getaffinity(0)),
+                   "kind": "oracle", "sample": desc, "seconds": secs}
+        clocks = clk.summary()
+        out = {"metric": METRIC, "value": world * wl.T / (ms * 1e-3), "unit": "tokens/s",
+               "n_gpus": world, "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms,
+               "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": wl.dtype,
+               "data": "synthetic (seeded SplitMix64 + Box-Muller normals; weights N(0, 1/fan_in))",
+               "config": config_of(wl), "roofline": roof, "layer_roofline": layer,
+               "cpu_baseline": cpu,
+               "e2e": {"value": world * wl.T / (e2e_ms * 1e-3), "unit": "tokens/s",
+                       "ms_per_step": e2e_ms,
+                       "h2d_bytes_per_step": int(xs[0].numel() * xs[0].element_size()),
+                       "d2h_bytes_per_step": int(y.numel() * y.element_size())},
+               "gpu_launches": int(launches),
+               "stages_ms": {k: v / max(1, nrec) for k, v in stages.items()},
+               "clocks": clocks, "input_gen_s": gen_s}
+    if dist is not None:
+        dist.barrier()
+        dist.destroy_process_group()
+    if out is not None:
+        print(json.dumps(out), flush=True)
+    return 0
+
+
+def wl_key(wl):
+    for k, v in synth.WORKLOADS.items():
+        if v == wl:
+            return k
+    return "custom"
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=200)
+    ap.add_argument("--warmup", type=int, default=10)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--workload", choices=list(synth.WORKLOADS), default="mixtral")
+    ap.add_argument("--cpu-budget", type=float, default=15.0,
+                    help="seconds of oracle work for the cpu_baseline sample")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    if args.warmup < 3:
+        ap.error("--warmup must be >= 3")
+    wl = synth.WORKLOADS[args.workload]
+    if args.impl == "reference":
+        return run_reference(args, wl)
+    return run_ours(args, wl)
+
+
+if __name__ == "__main__":
+    sys.exit(main())

@@ -305,3 +305,22 @@ def forward_rows_lazy(wl, x: np.ndarray, routing: dict, tokens, get_expert, shar
     if shared is not None:
         sh = dict(xsh=decode(xr), Ws1=shared[0], Ws3=shared[1], Ws2=shared[2])
     return layer_rows(wl.act, xin, lidx, gate, drop, W1, W3, W2, **sh)
+
+
+def combine(y_rows: np.ndarray, inv_row: np.ndarray, gate: np.ndarray, y_shared=None) -> np.ndarray:
+    """y[t] = sum over kept slots j of gate[t,j] * y_rows[inv_row[t*k+j]] (+ y_shared[t]).
+
+    "moe communication costs", Router design (weighted sum over the selected
+    experts); a dropped slot (inv_row = -1) contributes nothing.  fp64.
+    """
+    y_rows = np.asarray(y_rows, dtype=np.float64)
+    T, k = gate.shape
+    d = y_rows.shape[1]
+    rows = np.asarray(inv_row).reshape(T, k)
+    y = np.zeros((T, d))
+    for j in range(k):
+        m = rows[:, j] >= 0
+        y[m] += gate[m, j, None] * y_rows[rows[m, j]]
+    if y_shared is not None:
+        y += np.asarray(y_shared, dtype=np.float64)
+    return y

@@ -1,0 +1,95 @@
+"""C-ABI checks that need no GPU: the library loads, exports every function
+include/moe.h declares, and rejects bad arguments on the host before any
+launch."""
+import ctypes
+import os
+import re
+
+import pytest
+
+import top_routing_expert_warp_b200 as moe
+from top_routing_expert_warp_b200 import build as moe_build
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+@pytest.fixture(scope="module")
+def lib():
+    moe_build.build()
+    return moe.lib()
+
+
+def _declared():
+    txt = open(os.path.join(ROOT, "include", "moe.h")).read()
+    txt = re.sub(r"/\*.*?\*/", "", txt, flags=re.S)
+    return sorted(set(re.findall(r"\b(moe_[a-z_]+)\s*\(", txt)))
+
+
+def test_every_declared_symbol_is_exported(lib):
+    names = _declared()
+    assert "moe_layer_forward" in names and len(names) >= 10
+    for n in names:
+        assert hasattr(lib, n), n
+    assert set(names) <= set(moe.EXPORTS) | {"moe_layer_forward"}
+
+
+def test_version_and_status_strings(lib):
+    assert "sm_100a" in moe.moe_version()
+    assert moe.status_string(moe.MOE_OK) == "ok"
+    assert "workspace" in moe.status_string(moe.MOE_ERR_WORKSPACE)
+
+
+def test_workspace_bytes_and_config_validation(lib):
+    good = moe.make_config(4096, 4096, 8, 2, 14336)
+    n = moe.moe_workspace_bytes(good)
+    # x_perm + h + y_perm dominate: 8192 rows x (4096 + 14336 + 4096) bf16
+    assert n >= 8192 * (4096 + 14336 + 4096) * 2
+    assert n % 256 == 0
+    bad = [moe.make_config(16, 4096, 8, 9, 128),          # k > 8
+           moe.make_config(16, 4096, 4, 5, 128),          # k > N
+           moe.make_config(16, 4100, 8, 2, 128),          # d not a multiple of 8 (bf16)
+           moe.make_config(16, 64, 300, 2, 128),          # N > 256
+           moe.make_config(16, 64, 32, 2, 128, dtype="f32"),  # fp32 layers: N <= 16
+           moe.make_config(16, 64, 8, 2, 128, dtype="f32", dispatch_dtype="fp8")]
+    for c in bad:
+        assert moe.moe_workspace_bytes(c) == 0
+
+
+def test_entry_points_reject_bad_arguments_before_launch(lib):
+    cfg = moe.make_config(16, 64, 8, 2, 128)
+    nbytes = moe.moe_workspace_bytes(cfg)
+    P = ctypes.c_void_p
+    fake = 1 << 40          # never dereferenced: validation fails first
+    # null workspace
+    r = lib.moe_combine(ctypes.byref(cfg), P(fake), P(fake), P(fake), None, P(fake), None, nbytes, None)
+    assert r == moe.MOE_ERR_WORKSPACE
+    # misaligned workspace
+    r = lib.moe_combine(ctypes.byref(cfg), P(fake), P(fake), P(fake), None, P(fake), P(fake + 8),
+                        nbytes, None)
+    assert r == moe.MOE_ERR_WORKSPACE
+    # too small
+    r = lib.moe_combine(ctypes.byref(cfg), P(fake), P(fake), P(fake), None, P(fake), P(fake),
+                        nbytes - 256, None)
+    assert r == moe.MOE_ERR_WORKSPACE
+    # null required pointer
+    r = lib.moe_router(ctypes.byref(cfg), None, P(fake), None, None, P(fake), P(fake), None,
+                       P(fake), nbytes, None)
+    assert r == moe.MOE_ERR_INVALID_ARG
+    # misaligned activation
+    r = lib.moe_router(ctypes.byref(cfg), P(fake + 2), P(fake), None, None, P(fake), P(fake), None,
+                       P(fake), nbytes, None)
+    assert r == moe.MOE_ERR_INVALID_ARG
+    # aux loss without p_mean
+    r = lib.moe_dispatch(ctypes.byref(cfg), P(fake), P(fake), P(fake), P(fake), P(fake), P(fake),
+                         P(fake), P(fake), None, None, None, P(fake), P(fake), nbytes, None)
+    assert r == moe.MOE_ERR_INVALID_ARG
+    # FP8 dispatch without the scale buffer
+    c8 = moe.make_config(16, 64, 8, 2, 128, dispatch_dtype="fp8")
+    r = lib.moe_dispatch(ctypes.byref(c8), P(fake), P(fake), P(fake), P(fake), P(fake), P(fake),
+                         P(fake), P(fake), None, None, None, None, P(fake),
+                         moe.moe_workspace_bytes(c8), None)
+    assert r == moe.MOE_ERR_INVALID_ARG
+    # invalid config
+    badc = moe.make_config(16, 64, 8, 9, 128)
+    r = lib.moe_layer_forward(ctypes.byref(badc), *([None] * 17), 0, None)
+    assert r == moe.MOE_ERR_INVALID_ARG

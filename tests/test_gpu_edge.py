@@ -1,0 +1,123 @@
+"""Edge cases on the GPU: degenerate shapes, empty experts, full drops, T = 0,
+ragged tiles, and the device status word."""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+import synth
+import top_routing_expert_warp_b200 as moe
+from gpu_util import LayerRun, cfg_of, rel_l2, to_f64, upload_inputs, y_tol
+
+pytestmark = pytest.mark.gpu
+
+
+def _layer_vs_oracle(wl, tokens=None):
+    dev, host = upload_inputs(wl)
+    run = LayerRun(wl, dev)
+    run()
+    st = run.check_status()
+    assert st[0] == moe.MOE_OK, st
+    ref = oracle.route(wl, host["x"], host["Wg"], host.get("bias"))
+    assert np.array_equal(run.topk_idx.cpu().numpy(), ref["idx"])
+    tokens = np.arange(wl.T) if tokens is None else tokens
+    want = oracle.forward_rows(wl, host, ref, tokens)
+    got = to_f64(run.y)[tokens]
+    if np.abs(want).max() == 0:
+        assert np.all(got == 0)
+    else:
+        assert rel_l2(got, want) <= y_tol(wl)
+    return run, ref
+
+
+@pytest.mark.parametrize("base", [synth.TINY_F32, synth.MIXTRAL.with_(d=128, H=256),
+                                  synth.SWITCH.with_(d=128, H=256),
+                                  synth.DEEPSEEK.with_(d=128, H=128, H_shared=64)])
+def test_single_token(base):
+    _layer_vs_oracle(base.with_(T=1))
+
+
+@pytest.mark.parametrize("dtype", ["f32", "bf16"])
+def test_one_expert_k1_is_dense_ffn(dtype):
+    wl = synth.Workload("n1k1", T=129, d=64, N=1, k=1, H=256, act="swiglu", dtype=dtype,
+                        gate_mode="R", seed=21)
+    run, ref = _layer_vs_oracle(wl)
+    assert np.all(run.topk_w.cpu().numpy() == 1.0)
+
+
+def test_k_equals_n_full_softmax():
+    wl = synth.Workload("k=N", T=77, d=64, N=4, k=4, H=128, act="relu", dtype="bf16",
+                        gate_mode="R", seed=22)
+    _layer_vs_oracle(wl)
+
+
+def test_capacity_zero_drops_everything():
+    wl = synth.Workload("C=0", T=64, d=64, N=8, k=2, H=128, act="relu", dtype="bf16",
+                        gate_mode="F", capacity_factor=0.01, seed=23)
+    run, ref = _layer_vs_oracle(wl)
+    assert ref["R"] == 0
+    assert torch.all(run.y == 0)
+
+
+def test_empty_experts_large_n():
+    # a strong negative bias on half the experts leaves them without tokens
+    wl = synth.Workload("empty", T=300, d=128, N=64, k=2, H=128, act="swiglu", dtype="bf16",
+                        gate_mode="F", renormalize=True, bias_std=1.0, seed=24)
+    dev, host = upload_inputs(wl)
+    bias = host["bias"].copy()
+    bias[::2] = -100.0
+    dev["bias"] = torch.from_numpy(bias).cuda()
+    host["bias"] = bias
+    run = LayerRun(wl, dev)
+    run()
+    assert run.check_status()[0] == moe.MOE_OK
+    ref = oracle.route(wl, host["x"], host["Wg"], bias)
+    assert np.all(ref["counts"][::2] == 0)
+    assert np.array_equal(run.topk_idx.cpu().numpy(), ref["idx"])
+    want = oracle.forward_rows(wl, host, ref, np.arange(wl.T))
+    assert rel_l2(to_f64(run.y), want) <= y_tol(wl)
+
+
+def test_zero_tokens():
+    wl = synth.MIXTRAL.with_(T=0, d=128, H=128)
+    cfg = cfg_of(wl)
+    ws = moe.workspace(cfg)
+    dev, _ = upload_inputs(wl.with_(T=1))
+    y = torch.empty((0, wl.d), dtype=torch.bfloat16, device="cuda")
+    aux = torch.full((1,), 7.0, device="cuda")
+    pm = torch.full((wl.N,), 7.0, device="cuda")
+    moe.moe_layer_forward(cfg, dev["x"], dev["Wg"], None, dev["W1"], dev["W3"], dev["W2"],
+                          None, None, None, y, None, None, None, None, pm, aux, ws)
+    assert moe.moe_check_status(ws)[0] == moe.MOE_OK
+    assert aux.item() == 0.0 and torch.all(pm == 0)
+
+
+def test_bad_expert_index_sets_status_word():
+    wl = synth.MIXTRAL.with_(T=64, d=128, H=128)
+    cfg = cfg_of(wl)
+    ws = moe.workspace(cfg)
+    dev, _ = upload_inputs(wl)
+    idx = torch.from_numpy(synth.synthetic_topk(1, wl.T, wl.N, wl.k)).cuda()
+    idx[5, 1] = wl.N          # out of range
+    rows = wl.T * wl.k
+    counts = torch.empty(wl.N, dtype=torch.int32, device="cuda")
+    offs = torch.empty(wl.N + 1, dtype=torch.int32, device="cuda")
+    perm = torch.empty(rows, dtype=torch.int32, device="cuda")
+    inv = torch.empty(rows, dtype=torch.int32, device="cuda")
+    drop = torch.empty(rows, dtype=torch.uint8, device="cuda")
+    xp = torch.empty((rows, wl.d), dtype=torch.bfloat16, device="cuda")
+    moe.moe_dispatch(cfg, dev["x"], idx, counts, offs, perm, inv, drop, xp, None, None, None,
+                     None, ws)
+    st, word = moe.moe_check_status(ws)
+    assert st == moe.MOE_ERR_DEVICE_STATUS and (word & 1)
+    assert drop[5 * wl.k + 1].item() == 1 and inv[5 * wl.k + 1].item() == -1
+    assert counts.sum().item() == rows - 1
+    # the word was cleared by the read
+    assert moe.moe_check_status(ws) == (moe.MOE_OK, 0)
+
+
+def test_ragged_rows_many_tiles():
+    # 1 expert, 3 m-tiles with a ragged tail, two SwiGLU n-tiles
+    wl = synth.Workload("ragged", T=300, d=192, N=1, k=1, H=256, act="swiglu", dtype="bf16",
+                        gate_mode="R", seed=25)
+    _layer_vs_oracle(wl)

@@ -121,3 +121,19 @@ def test_lazy_rows_equal_stacked_rows():
     b = oracle.forward_rows_lazy(wl, inp["x"], routing, toks,
                                  lambda e: (inp["W1"][e], inp["W3"][e], inp["W2"][e]))
     assert np.array_equal(a, b)
+
+
+def test_combine_bruteforce():
+    T, k, d = 17, 3, 5
+    rng_rows = synth.normal(1, 40, 30 * d, 1.0, "f32").reshape(30, d).astype(np.float64)
+    inv = synth.uniform_int(2, 41, T * k, 31) - 1          # -1 .. 29
+    gate = synth.normal(3, 42, T * k, 1.0, "f32").reshape(T, k).astype(np.float64)
+    ysh = synth.normal(4, 43, T * d, 1.0, "f32").reshape(T, d).astype(np.float64)
+    y = oracle.combine(rng_rows, inv, gate, ysh)
+    for t in range(T):
+        ref = ysh[t].copy()
+        for j in range(k):
+            r = inv[t * k + j]
+            if r >= 0:
+                ref = ref + gate[t, j] * rng_rows[r]
+        np.testing.assert_allclose(y[t], ref, rtol=1e-14, atol=1e-14)

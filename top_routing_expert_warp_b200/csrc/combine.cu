@@ -1,0 +1,144 @@
+// Combine: the gate-weighted un-permute.
+//
+//   y[t] = sum over kept slots j (in slot order) of g[t, j] * y_perm[inv_row[t k + j]]
+//          (+ y_shared[t])
+//
+// "moe communication costs", Router design: the layer output is the sum over
+// the selected experts of G(x)_i E_i(x); on one GPU the return all-to-all of
+// "MoE: what it costs to train and serve" (Expert parallelism, step 3) becomes
+// this gather.  A dropped slot (inv_row = -1, "moe communication costs",
+// Capacity factor) contributes nothing.  The always-on shared expert's output,
+// when present, is added with coefficient 1.  One warp per token, 16-byte
+// accesses, fp32 accumulation in a fixed order.
+#include "common.cuh"
+#include "kernels.h"
+#include "moe.h"
+
+namespace moe {
+
+namespace {
+
+constexpr int kThreads = 256;
+constexpr int kWarps = kThreads / 32;
+constexpr int kMaxK = 8;
+
+template <bool BF16>
+__global__ void __launch_bounds__(kThreads)
+    combine_kernel(const uint8_t *__restrict__ y_perm, const int32_t *__restrict__ inv_row,
+                   const float *__restrict__ topk_w, const uint8_t *__restrict__ y_shared,
+                   uint8_t *__restrict__ y, int64_t T, int d, int k, int64_t rows_cap,
+                   uint32_t *status)
+{
+    const int lane = threadIdx.x & 31;
+    const int esz = BF16 ? 2 : 4;
+    const int chunks = d * esz / 16;
+    const int64_t nwarps = static_cast<int64_t>(gridDim.x) * kWarps;
+    for (int64_t t = static_cast<int64_t>(blockIdx.x) * kWarps + (threadIdx.x >> 5); t < T;
+         t += nwarps) {
+        int32_t row[kMaxK];
+        float g[kMaxK];
+        int32_t my_row = -1;
+        float my_g = 0.0f;
+        if (lane < k) {
+            my_row = inv_row[t * k + lane];
+            my_g = topk_w[t * k + lane];
+            if (my_row >= rows_cap || my_row < -1) {
+                set_status(status, DEV_BAD_ROW);
+                my_row = -1;
+            }
+        }
+#pragma unroll
+        for (int j = 0; j < kMaxK; ++j) {
+            row[j] = __shfl_sync(0xffffffffu, my_row, j);
+            g[j] = __shfl_sync(0xffffffffu, my_g, j);
+        }
+        for (int c = lane; c < chunks; c += 32) {
+            constexpr int V = BF16 ? 8 : 4;
+            float acc[V];
+#pragma unroll
+            for (int i = 0; i < V; ++i)
+                acc[i] = 0.0f;
+#pragma unroll
+            for (int j = 0; j < kMaxK; ++j) {
+                if (j < k && row[j] >= 0) {
+                    const uint4 v = __ldg(reinterpret_cast<const uint4 *>(
+                                              y_perm + static_cast<int64_t>(row[j]) * d * esz) +
+                                          c);
+                    const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+                    if (BF16) {
+#pragma unroll
+                        for (int i = 0; i < 4; ++i) {
+                            acc[2 * i] = fmaf(g[j], __uint_as_float(w[i] << 16), acc[2 * i]);
+                            acc[2 * i + 1] =
+                                fmaf(g[j], __uint_as_float(w[i] & 0xFFFF0000u), acc[2 * i + 1]);
+                        }
+                    } else {
+#pragma unroll
+                        for (int i = 0; i < 4; ++i)
+                            acc[i] = fmaf(g[j], __uint_as_float(w[i]), acc[i]);
+                    }
+                }
+            }
+            if (y_shared != nullptr) {
+                const uint4 v = __ldg(
+                    reinterpret_cast<const uint4 *>(y_shared + t * static_cast<int64_t>(d) * esz) + c);
+                const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+                if (BF16) {
+#pragma unroll
+                    for (int i = 0; i < 4; ++i) {
+                        acc[2 * i] += __uint_as_float(w[i] << 16);
+                        acc[2 * i + 1] += __uint_as_float(w[i] & 0xFFFF0000u);
+                    }
+                } else {
+#pragma unroll
+                    for (int i = 0; i < 4; ++i)
+                        acc[i] += __uint_as_float(w[i]);
+                }
+            }
+            uint4 o;
+            if (BF16) {
+                o.x = pack_bf16x2(acc[0], acc[1]);
+                o.y = pack_bf16x2(acc[2], acc[3]);
+                o.z = pack_bf16x2(acc[4], acc[5]);
+                o.w = pack_bf16x2(acc[6], acc[7]);
+            } else {
+                o.x = __float_as_uint(acc[0]);
+                o.y = __float_as_uint(acc[1]);
+                o.z = __float_as_uint(acc[2]);
+                o.w = __float_as_uint(acc[3]);
+            }
+            reinterpret_cast<uint4 *>(y + t * static_cast<int64_t>(d) * esz)[c] = o;
+        }
+    }
+}
+
+}  // namespace
+
+cudaError_t launch_combine(int dtype, const void *y_perm, const int32_t *inv_row,
+                           const float *topk_w, const void *y_shared, void *y, int64_t T,
+                           int32_t d, int32_t k, uint32_t *status, cudaStream_t stream)
+{
+    if (T == 0)
+        return cudaSuccess;
+    int sms = 148, dev = 0;
+    if (cudaGetDevice(&dev) == cudaSuccess)
+        cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+    int64_t grid = (T + kWarps - 1) / kWarps;
+    if (grid > static_cast<int64_t>(sms) * 8)
+        grid = static_cast<int64_t>(sms) * 8;
+    const int64_t rows_cap = T * k;
+    if (dtype == MOE_BF16)
+        combine_kernel<true><<<static_cast<int>(grid), kThreads, 0, stream>>>(
+            static_cast<const uint8_t *>(y_perm), inv_row, topk_w,
+            static_cast<const uint8_t *>(y_shared), static_cast<uint8_t *>(y), T, d, k, rows_cap,
+            status);
+    else
+        combine_kernel<false><<<static_cast<int>(grid), kThreads, 0, stream>>>(
+            static_cast<const uint8_t *>(y_perm), inv_row, topk_w,
+            static_cast<const uint8_t *>(y_shared), static_cast<uint8_t *>(y), T, d, k, rows_cap,
+            status);
+    count_launches(1);
+    return cudaGetLastError();
+}
+
+}  // namespace moe

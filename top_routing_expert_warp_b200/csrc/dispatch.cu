@@ -1,0 +1,361 @@
+// Dispatch as an on-device permutation of (token, slot) pairs into
+// expert-contiguous rows.
+//
+// On one GPU the first all-to-all of the expert-parallel flow ("MoE: what it
+// costs to train and serve", Expert parallelism and two all-to-alls, step 1)
+// becomes a counting sort of the pairs by expert.  Capacity follows "moe
+// communication costs", Capacity factor and token dropping: expert e keeps
+// at most C = floor(capacity_factor * T / N) pairs, the first C in token
+// order; the rest are dropped.  The aux-loss statistics follow the same
+// page's Load balancing paragraph: f_i = pairs routed to i (before dropping)
+// / (T k), L_aux = alpha N sum_i f_i p_i.
+//
+// Kernels (one stream, no host synchronisation):
+//   count  - per block of 2048 pairs, per-expert counts with warp-aggregated
+//            shared-memory atomics (__match_any_sync groups equal experts);
+//   scan   - one block: per expert, exclusive scan over blocks (block bases),
+//            counts, kept = min(count, C), offsets = exclusive scan of kept,
+//            f and L_aux in a fixed summation order;
+//   rank   - stable rank of every pair inside its expert: block base +
+//            earlier warps of the block + earlier lanes of the warp; writes
+//            perm / inv_row / drop;
+//   gather - one warp per kept row copies x[token] with 16-byte accesses,
+//            or quantises it to FP8 E4M3 with a per-row fp32 scale
+//            (amax / 448) as the page's FP8 dispatch payload does ("MoE: what
+//            it costs to train and serve", Worked example: bytes per token).
+#include <cuda_fp8.h>
+
+#include "common.cuh"
+#include "kernels.h"
+#include "moe.h"
+
+namespace moe {
+
+namespace {
+
+constexpr int kThreads = 256;
+constexpr int kWarps = kThreads / 32;
+constexpr int kPerWarp = kDispChunk / kWarps;  // 256 pairs, 8 rounds of 32
+
+__global__ void __launch_bounds__(kThreads)
+    dispatch_count_kernel(const int32_t *__restrict__ idx, int64_t n_pairs, int N,
+                          int32_t *__restrict__ block_base, uint32_t *status)
+{
+    extern __shared__ int32_t s_cnt[];
+    for (int e = threadIdx.x; e < N; e += kThreads)
+        s_cnt[e] = 0;
+    __syncthreads();
+    const int lane = threadIdx.x & 31;
+    const int64_t base = static_cast<int64_t>(blockIdx.x) * kDispChunk;
+    for (int r = 0; r < kDispChunk / kThreads; ++r) {
+        const int64_t i = base + r * kThreads + threadIdx.x;
+        int e = -1;
+        if (i < n_pairs) {
+            e = idx[i];
+            if (e < 0 || e >= N) {
+                set_status(status, DEV_BAD_EXPERT);
+                e = -1;
+            }
+        }
+        const uint32_t peers = __match_any_sync(0xffffffffu, e);
+        if (e >= 0 && lane == __ffs(peers) - 1)
+            atomicAdd(&s_cnt[e], __popc(peers));
+    }
+    __syncthreads();
+    for (int e = threadIdx.x; e < N; e += kThreads)
+        block_base[static_cast<int64_t>(blockIdx.x) * N + e] = s_cnt[e];
+}
+
+__global__ void __launch_bounds__(1024)
+    dispatch_scan_kernel(int nblk, int N, int64_t n_pairs, int64_t C,
+                         int32_t *__restrict__ block_base, int32_t *__restrict__ counts,
+                         int32_t *__restrict__ offsets, const float *__restrict__ p_mean,
+                         float *__restrict__ f, float *__restrict__ aux_loss, float alpha)
+{
+    __shared__ int32_t s_warp[32];
+    __shared__ double s_aux[1024];
+    const int e = threadIdx.x;
+    const int lane = e & 31, warp = e >> 5;
+    int32_t kept = 0;
+    int32_t run = 0;
+    if (e < N) {
+        for (int b = 0; b < nblk; ++b) {
+            const int64_t o = static_cast<int64_t>(b) * N + e;
+            const int32_t v = block_base[o];
+            block_base[o] = run;
+            run += v;
+        }
+        counts[e] = run;
+        kept = (C >= 0 && run > C) ? static_cast<int32_t>(C) : run;
+        if (f != nullptr)
+            f[e] = static_cast<float>(static_cast<double>(run) / static_cast<double>(n_pairs));
+    }
+    // exclusive scan of kept over experts
+    int32_t incl = kept;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+        const int32_t v = __shfl_up_sync(0xffffffffu, incl, o);
+        if (lane >= o)
+            incl += v;
+    }
+    if (lane == 31)
+        s_warp[warp] = incl;
+    __syncthreads();
+    if (warp == 0) {
+        int32_t w = s_warp[lane];
+        int32_t wi = w;
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+            const int32_t v = __shfl_up_sync(0xffffffffu, wi, o);
+            if (lane >= o)
+                wi += v;
+        }
+        s_warp[lane] = wi - w;  // exclusive warp base
+    }
+    __syncthreads();
+    const int32_t excl = s_warp[warp] + incl - kept;
+    if (e < N)
+        offsets[e] = excl;
+    if (e == N - 1)
+        offsets[N] = excl + kept;
+    // L_aux = alpha N sum_e f_e p_e, summed in a fixed tree order
+    if (aux_loss != nullptr && p_mean != nullptr) {
+        double term = 0.0;
+        if (e < N)
+            term = static_cast<double>(run) / static_cast<double>(n_pairs) *
+                   static_cast<double>(p_mean[e]);
+        s_aux[e] = term;
+        __syncthreads();
+        for (int s = 512; s > 0; s >>= 1) {
+            if (e < s)
+                s_aux[e] += s_aux[e + s];
+            __syncthreads();
+        }
+        if (e == 0)
+            *aux_loss = static_cast<float>(static_cast<double>(alpha) * N * s_aux[0]);
+    }
+}
+
+__global__ void __launch_bounds__(kThreads)
+    dispatch_rank_kernel(const int32_t *__restrict__ idx, int64_t n_pairs, int N, int64_t C,
+                         const int32_t *__restrict__ block_base,
+                         const int32_t *__restrict__ offsets, int32_t *__restrict__ perm,
+                         int32_t *__restrict__ inv_row, uint8_t *__restrict__ drop)
+{
+    extern __shared__ int32_t s_w[];  // [kWarps][N]
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    for (int i = threadIdx.x; i < kWarps * N; i += kThreads)
+        s_w[i] = 0;
+    __syncthreads();
+    const int64_t wbase = static_cast<int64_t>(blockIdx.x) * kDispChunk + warp * kPerWarp;
+    int32_t *mine = s_w + warp * N;
+    // phase 1: per-warp counts
+    for (int r = 0; r < kPerWarp / 32; ++r) {
+        const int64_t i = wbase + r * 32 + lane;
+        int e = -1;
+        if (i < n_pairs) {
+            e = idx[i];
+            if (e < 0 || e >= N)
+                e = -1;
+        }
+        const uint32_t peers = __match_any_sync(0xffffffffu, e);
+        if (e >= 0 && lane == __ffs(peers) - 1)
+            mine[e] += __popc(peers);
+        __syncwarp();
+    }
+    __syncthreads();
+    // phase 2: warp bases = block base + counts of earlier warps
+    for (int e = threadIdx.x; e < N; e += kThreads) {
+        int32_t run = block_base[static_cast<int64_t>(blockIdx.x) * N + e];
+        for (int w = 0; w < kWarps; ++w) {
+            const int32_t v = s_w[w * N + e];
+            s_w[w * N + e] = run;
+            run += v;
+        }
+    }
+    __syncthreads();
+    // phase 3: walk the pairs in order; rank = warp base + earlier lanes
+    for (int r = 0; r < kPerWarp / 32; ++r) {
+        const int64_t i = wbase + r * 32 + lane;
+        int e = -1;
+        if (i < n_pairs) {
+            e = idx[i];
+            if (e < 0 || e >= N)
+                e = -1;
+        }
+        const uint32_t peers = __match_any_sync(0xffffffffu, e);
+        int32_t rank = 0;
+        if (e >= 0)
+            rank = mine[e] + __popc(peers & lanemask_lt());
+        __syncwarp();
+        if (e >= 0 && lane == __ffs(peers) - 1)
+            mine[e] += __popc(peers);
+        __syncwarp();
+        if (i < n_pairs) {
+            if (e < 0 || (C >= 0 && rank >= C)) {
+                drop[i] = 1;
+                inv_row[i] = -1;
+            } else {
+                const int32_t row = offsets[e] + rank;
+                perm[row] = static_cast<int32_t>(i);
+                inv_row[i] = row;
+                drop[i] = 0;
+            }
+        }
+    }
+}
+
+// One warp per kept row.  BF16 in -> copy (or FP8 quantise); F32 in -> copy.
+template <bool BF16, bool FP8>
+__global__ void __launch_bounds__(kThreads)
+    dispatch_gather_kernel(const uint8_t *__restrict__ x, int d, int k,
+                           const int32_t *__restrict__ perm, const int32_t *__restrict__ R_ptr,
+                           uint8_t *__restrict__ x_perm, float *__restrict__ x_scale,
+                           __nv_bfloat16 *__restrict__ x_bf16_copy)
+{
+    const int lane = threadIdx.x & 31;
+    const int64_t R = *R_ptr;
+    const int64_t nwarps = static_cast<int64_t>(gridDim.x) * kWarps;
+    const int esz = BF16 ? 2 : 4;
+    const int chunks = d * esz / 16;
+    for (int64_t r = static_cast<int64_t>(blockIdx.x) * kWarps + (threadIdx.x >> 5); r < R;
+         r += nwarps) {
+        const int64_t t = perm[r] / k;
+        const uint4 *src = reinterpret_cast<const uint4 *>(x + t * static_cast<int64_t>(d) * esz);
+        if (!FP8) {
+            uint4 *dst = reinterpret_cast<uint4 *>(x_perm + r * static_cast<int64_t>(d) * esz);
+            for (int c = lane; c < chunks; c += 32)
+                dst[c] = __ldg(src + c);
+        } else {
+            float amax = 0.0f;
+            for (int c = lane; c < chunks; c += 32) {
+                const uint4 v = __ldg(src + c);
+                const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+                for (int i = 0; i < 4; ++i) {
+                    amax = fmaxf(amax, fabsf(__uint_as_float(w[i] << 16)));
+                    amax = fmaxf(amax, fabsf(__uint_as_float(w[i] & 0xFFFF0000u)));
+                }
+            }
+#pragma unroll
+            for (int o = 16; o > 0; o >>= 1)
+                amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, o));
+            const float scale = amax > 0.0f ? __fdiv_rn(amax, 448.0f) : 1.0f;
+            if (lane == 0)
+                x_scale[r] = scale;
+            uint2 *dq = reinterpret_cast<uint2 *>(x_perm + r * static_cast<int64_t>(d));
+            uint4 *db = x_bf16_copy
+                            ? reinterpret_cast<uint4 *>(x_bf16_copy + r * static_cast<int64_t>(d))
+                            : nullptr;
+            for (int c = lane; c < chunks; c += 32) {
+                const uint4 v = __ldg(src + c);
+                const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+                uint32_t q[2] = {0u, 0u};
+                uint32_t b[4];
+#pragma unroll
+                for (int i = 0; i < 4; ++i) {
+                    const float lo = __fdiv_rn(__uint_as_float(w[i] << 16), scale);
+                    const float hi = __fdiv_rn(__uint_as_float(w[i] & 0xFFFF0000u), scale);
+                    const __nv_fp8_storage_t qlo = __nv_cvt_float_to_fp8(lo, __NV_SATFINITE, __NV_E4M3);
+                    const __nv_fp8_storage_t qhi = __nv_cvt_float_to_fp8(hi, __NV_SATFINITE, __NV_E4M3);
+                    q[i >> 1] |= (static_cast<uint32_t>(qlo) | (static_cast<uint32_t>(qhi) << 8))
+                                 << (16 * (i & 1));
+                    if (db) {
+                        __nv_fp8_e4m3 flo, fhi;
+                        flo.__x = qlo;
+                        fhi.__x = qhi;
+                        b[i] = pack_bf16x2(static_cast<float>(flo), static_cast<float>(fhi));
+                    }
+                }
+                dq[c] = make_uint2(q[0], q[1]);
+                if (db)
+                    db[c] = make_uint4(b[0], b[1], b[2], b[3]);
+            }
+        }
+    }
+}
+
+__global__ void __launch_bounds__(kThreads)
+    fp8_to_bf16_kernel(const uint8_t *__restrict__ q, int d, const int32_t *__restrict__ R_ptr,
+                       __nv_bfloat16 *__restrict__ out)
+{
+    const int lane = threadIdx.x & 31;
+    const int64_t R = *R_ptr;
+    const int64_t nwarps = static_cast<int64_t>(gridDim.x) * kWarps;
+    const int chunks = d / 8;
+    for (int64_t r = static_cast<int64_t>(blockIdx.x) * kWarps + (threadIdx.x >> 5); r < R;
+         r += nwarps) {
+        const uint2 *src = reinterpret_cast<const uint2 *>(q + r * static_cast<int64_t>(d));
+        uint4 *dst = reinterpret_cast<uint4 *>(out + r * static_cast<int64_t>(d));
+        for (int c = lane; c < chunks; c += 32) {
+            const uint2 v = src[c];
+            const uint32_t w[2] = {v.x, v.y};
+            uint32_t b[4];
+#pragma unroll
+            for (int i = 0; i < 4; ++i) {
+                __nv_fp8_e4m3 lo, hi;
+                lo.__x = static_cast<__nv_fp8_storage_t>((w[i >> 1] >> (16 * (i & 1))) & 0xFF);
+                hi.__x = static_cast<__nv_fp8_storage_t>((w[i >> 1] >> (16 * (i & 1) + 8)) & 0xFF);
+                b[i] = pack_bf16x2(static_cast<float>(lo), static_cast<float>(hi));
+            }
+            dst[c] = make_uint4(b[0], b[1], b[2], b[3]);
+        }
+    }
+}
+
+int gather_grid(int64_t rows)
+{
+    int sms = 148, dev = 0;
+    if (cudaGetDevice(&dev) == cudaSuccess)
+        cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+    int64_t want = (rows + kWarps - 1) / kWarps;
+    const int64_t cap = static_cast<int64_t>(sms) * 8;
+    if (want > cap)
+        want = cap;
+    return want < 1 ? 1 : static_cast<int>(want);
+}
+
+}  // namespace
+
+cudaError_t launch_dispatch(const DispatchLaunch &L, cudaStream_t stream)
+{
+    const int64_t n_pairs = L.T * L.k;
+    if (n_pairs == 0)
+        return cudaSuccess;
+    const int nblk = static_cast<int>((n_pairs + kDispChunk - 1) / kDispChunk);
+    dispatch_count_kernel<<<nblk, kThreads, L.N * sizeof(int32_t), stream>>>(
+        L.topk_idx, n_pairs, L.N, L.block_base, L.status);
+    dispatch_scan_kernel<<<1, 1024, 0, stream>>>(nblk, L.N, n_pairs, L.capacity, L.block_base,
+                                                 L.counts, L.offsets, L.p_mean, L.f, L.aux_loss,
+                                                 L.aux_alpha);
+    dispatch_rank_kernel<<<nblk, kThreads, kWarps * L.N * sizeof(int32_t), stream>>>(
+        L.topk_idx, n_pairs, L.N, L.capacity, L.block_base, L.offsets, L.perm, L.inv_row, L.drop);
+    const int grid = gather_grid(n_pairs);
+    const uint8_t *x = static_cast<const uint8_t *>(L.x);
+    uint8_t *xp = static_cast<uint8_t *>(L.x_perm);
+    if (L.dtype == MOE_F32)
+        dispatch_gather_kernel<false, false><<<grid, kThreads, 0, stream>>>(
+            x, L.d, L.k, L.perm, L.offsets + L.N, xp, nullptr, nullptr);
+    else if (!L.fp8)
+        dispatch_gather_kernel<true, false><<<grid, kThreads, 0, stream>>>(
+            x, L.d, L.k, L.perm, L.offsets + L.N, xp, nullptr, nullptr);
+    else
+        dispatch_gather_kernel<true, true><<<grid, kThreads, 0, stream>>>(
+            x, L.d, L.k, L.perm, L.offsets + L.N, xp, L.x_scale,
+            static_cast<__nv_bfloat16 *>(L.x_bf16_copy));
+    count_launches(4);
+    return cudaGetLastError();
+}
+
+cudaError_t launch_fp8_to_bf16(const uint8_t *q, int64_t rows_cap, int32_t d,
+                               const int32_t *offsets, int32_t N, void *out, cudaStream_t stream)
+{
+    if (rows_cap == 0)
+        return cudaSuccess;
+    fp8_to_bf16_kernel<<<gather_grid(rows_cap), kThreads, 0, stream>>>(
+        q, d, offsets + N, static_cast<__nv_bfloat16 *>(out));
+    count_launches(1);
+    return cudaGetLastError();
+}
+
+}  // namespace moe

@@ -1,0 +1,513 @@
+// Grouped GEMM on the 5th-generation tensor cores (tcgen05 + TMEM + TMA).
+//
+// Computes, for every group g (an expert's row segment),
+//   D[r, n] = epilogue( sum_k A[r, k] * B[g * n_out + n, k] )
+// for rows r in [offsets[g], offsets[g+1]) and n in [0, n_out).  A and B are
+// bf16, K-major (the reduction axis contiguous), accumulation is fp32 in TMEM.
+//
+// This one kernel serves every dense contraction of the MoE layer forward:
+//   - the router logits x W_g^T (one group, fp32 output; "moe communication
+//     costs", Router design),
+//   - the expert up-projection with a fused ReLU or SwiGLU epilogue and the
+//     down-projection ("MoE: what it costs to train and serve", Expert
+//     parallelism step 2, run locally), and the shared expert.
+//
+// Design (sm_100a):
+//   - persistent CTAs, one per SM, walking a static round-robin tile list;
+//     the tile list is derived on the device from the group offsets, so no
+//     host synchronisation is needed between dispatch and the GEMM;
+//   - tile = 128 rows x BN columns of the MMA (BN <= 256), K step 64 (one
+//     128-byte swizzle atom of bf16); for SwiGLU the BN = 256 MMA columns hold
+//     128 columns of W1 next to the same 128 columns of W3, so one MMA feeds
+//     both halves of the gated activation;
+//   - warp 0: TMA producer (one thread); warp 1: TMEM allocator and MMA issuer
+//     (one thread); warps 2-5: epilogue, one TMEM lane quarter each;
+//   - an S-stage shared-memory ring (full/empty mbarriers) and two TMEM
+//     accumulators, so the epilogue of one tile overlaps the MMAs of the next;
+//   - tile order inside a group: m fastest, so CTAs running at the same time
+//     share the weight tile through L2;
+//   - every mbarrier wait is bounded in time; on expiry the kernel records a
+//     status bit, tells the other roles to stop, waits (bounded) for its own
+//     copies and MMAs in flight, frees TMEM and returns.
+#include "common.cuh"
+#include "kernels.h"
+
+namespace moe {
+
+namespace {
+
+constexpr int BM = 128;
+constexpr int BK = 64;                      // bf16 elements per 128-byte row
+constexpr int A_STAGE_BYTES = BM * BK * 2;  // 16 KB
+constexpr int kThreads = 192;
+constexpr int kMaxGroups = 1024;
+
+struct GemmParams {
+    const int32_t *offsets;  // [G+1] row offsets of the groups in A, or null
+    int32_t rows_single;     // rows of the only group when offsets is null
+    int32_t G;
+    int32_t n_out;           // output columns per group (= rows of B per group)
+    int32_t K;
+    void *out;
+    int64_t ld_out;          // elements
+    const float *row_scale;  // multiply each accumulator row by row_scale[r], or null
+    int64_t rows_cap;        // rows allocated in out (and row_scale); rows beyond are never written
+    uint32_t *status;
+};
+
+template <int BN, int EPI>
+struct Geometry {
+    static constexpr int OUTN = (EPI == EPI_SWIGLU) ? BN / 2 : BN;
+    static constexpr int B_STAGE_BYTES = BN * BK * 2;
+    static constexpr int STAGE_BYTES = A_STAGE_BYTES + B_STAGE_BYTES;
+    static constexpr int STAGES = (BN >= 256) ? 4 : ((BN >= 128) ? 6 : 8);
+    static constexpr int TMEM_COLS = (2 * BN <= 32) ? 32 : (2 * BN <= 64 ? 64 : (2 * BN <= 128 ? 128 : (2 * BN <= 256 ? 256 : 512)));
+    // shared memory: [1 KB align slack][stages][barriers + tables]
+    static constexpr int AUX_BYTES = 8 * (2 * STAGES + 5) + 16 + 8 * (kMaxGroups + 2);
+    static constexpr int SMEM_BYTES = 1024 + STAGES * STAGE_BYTES + AUX_BYTES;
+};
+
+struct TileInfo {
+    int32_t g, row0, rows_valid, n0;
+};
+
+// Locate tile t: prefix[g] <= t < prefix[g+1].
+__device__ __forceinline__ TileInfo tile_info(int t, const int32_t *s_prefix,
+                                              const int32_t *s_off, int G, int n_tiles,
+                                              int outn)
+{
+    int lo = 0, hi = G;  // find largest g with prefix[g] <= t
+    while (hi - lo > 1) {
+        int mid = (lo + hi) >> 1;
+        if (s_prefix[mid] <= t)
+            lo = mid;
+        else
+            hi = mid;
+    }
+    int g = lo;
+    int rows_g = s_off[g + 1] - s_off[g];
+    int mt_g = (rows_g + BM - 1) / BM;
+    int local = t - s_prefix[g];
+    int n_tile = local / mt_g;
+    int m_tile = local - n_tile * mt_g;
+    TileInfo ti;
+    ti.g = g;
+    ti.row0 = s_off[g] + m_tile * BM;
+    ti.rows_valid = min(BM, rows_g - m_tile * BM);
+    ti.n0 = n_tile * outn;
+    (void)n_tiles;
+    return ti;
+}
+
+__device__ __forceinline__ float silu_f(float a)
+{
+    return a / (1.0f + __expf(-a));
+}
+
+template <int BN, int EPI, bool OUT_F32>
+__global__ void __launch_bounds__(kThreads, 1)
+    grouped_gemm_tc(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
+                    const __grid_constant__ CUtensorMap tmB2, GemmParams p)
+{
+    using Geo = Geometry<BN, EPI>;
+    constexpr int STAGES = Geo::STAGES;
+    constexpr int OUTN = Geo::OUTN;
+
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
+                                                ~static_cast<uintptr_t>(1023));
+    uint8_t *stage_base = smem;
+    uint64_t *bars = reinterpret_cast<uint64_t *>(smem + STAGES * Geo::STAGE_BYTES);
+    uint64_t *full = bars;
+    uint64_t *empty = bars + STAGES;
+    uint64_t *acc_full = bars + 2 * STAGES;
+    uint64_t *acc_empty = bars + 2 * STAGES + 2;
+    uint64_t *drain = bars + 2 * STAGES + 4;
+    uint32_t *s_tmem = reinterpret_cast<uint32_t *>(bars + 2 * STAGES + 5);
+    volatile int *s_abort = reinterpret_cast<volatile int *>(s_tmem + 1);
+    int32_t *s_off = reinterpret_cast<int32_t *>(s_tmem + 4);
+    int32_t *s_prefix = s_off + (kMaxGroups + 1);
+
+    const int warp = threadIdx.x >> 5;
+    const int lane = threadIdx.x & 31;
+    const int G = p.G;
+    const int n_tiles = (p.n_out + OUTN - 1) / OUTN;
+    const int KB = (p.K + BK - 1) / BK;
+
+    // ---- group table and tile prefix (warp 2), barriers (warp 0), TMEM (warp 1)
+    if (warp == 0 && lane == 0) {
+        for (int s = 0; s < STAGES; ++s) {
+            mbar_init(&full[s], 1);
+            mbar_init(&empty[s], 1);
+        }
+        for (int a = 0; a < 2; ++a) {
+            mbar_init(&acc_full[a], 1);
+            mbar_init(&acc_empty[a], 4 * 32);
+        }
+        mbar_init(drain, 1);
+        *s_abort = 0;
+        fence_barrier_init();
+        tma_prefetch_desc(&tmA);
+        tma_prefetch_desc(&tmB);
+        if (EPI == EPI_SWIGLU)
+            tma_prefetch_desc(&tmB2);
+    }
+    if (warp == 1) {
+        tmem_alloc(s_tmem, Geo::TMEM_COLS);
+        tmem_relinquish();
+    }
+    if (warp == 2) {
+        // offsets -> smem; per-group tile counts -> inclusive scan over groups
+        const int per = (G + 32) / 32;  // G+1 entries of offsets
+        for (int i = lane; i <= G; i += 32)
+            s_off[i] = p.offsets ? p.offsets[i] : (i == 0 ? 0 : p.rows_single);
+        __syncwarp();
+        int base = lane * per, sum = 0;
+        for (int i = 0; i < per; ++i) {
+            int g = base + i;
+            if (g < G) {
+                int rows = s_off[g + 1] - s_off[g];
+                rows = rows > 0 ? rows : 0;
+                sum += ((rows + BM - 1) / BM) * n_tiles;
+            }
+        }
+        int incl = sum;
+        for (int o = 1; o < 32; o <<= 1) {
+            int v = __shfl_up_sync(0xffffffffu, incl, o);
+            if (lane >= o)
+                incl += v;
+        }
+        int run = incl - sum;
+        for (int i = 0; i < per; ++i) {
+            int g = base + i;
+            if (g <= G) {
+                s_prefix[g] = run;
+                if (g < G) {
+                    int rows = s_off[g + 1] - s_off[g];
+                    rows = rows > 0 ? rows : 0;
+                    run += ((rows + BM - 1) / BM) * n_tiles;
+                }
+            }
+        }
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem_base = *s_tmem;
+    const int total_tiles = s_prefix[G];
+
+    if (warp == 0) {
+        // ================= TMA producer =================
+        if (lane == 0) {
+            int s = 0;
+            uint32_t ph = 0;
+            uint32_t last_par[STAGES];
+            uint32_t used = 0;
+            bool ok = true;
+            for (int t = blockIdx.x; t < total_tiles && ok; t += gridDim.x) {
+                TileInfo ti = tile_info(t, s_prefix, s_off, G, n_tiles, OUTN);
+                const int brow = ti.g * p.n_out + ti.n0;
+                for (int kb = 0; kb < KB; ++kb) {
+                    if (!mbar_wait_bounded(&empty[s], ph ^ 1u, s_abort)) {
+                        set_status(p.status, DEV_TIMEOUT_PRODUCER);
+                        *s_abort = 1;
+                        ok = false;
+                        break;
+                    }
+                    uint8_t *sa = stage_base + s * Geo::STAGE_BYTES;
+                    uint8_t *sb = sa + A_STAGE_BYTES;
+                    mbar_arrive_expect_tx(&full[s], Geo::STAGE_BYTES);
+                    tma_load_2d(sa, &tmA, &full[s], kb * BK, ti.row0);
+                    if (EPI == EPI_SWIGLU) {
+                        tma_load_2d(sb, &tmB, &full[s], kb * BK, brow);
+                        tma_load_2d(sb + (BN / 2) * BK * 2, &tmB2, &full[s], kb * BK, brow);
+                    } else {
+                        tma_load_2d(sb, &tmB, &full[s], kb * BK, brow);
+                    }
+                    last_par[s] = ph;
+                    used |= 1u << s;
+                    if (++s == STAGES) {
+                        s = 0;
+                        ph ^= 1u;
+                    }
+                }
+            }
+            // copies still in flight land before the CTA may exit
+            for (int i = 0; i < STAGES; ++i) {
+                if ((used >> i) & 1u) {
+                    volatile int never = 0;
+                    if (!mbar_wait_bounded(&full[i], last_par[i], &never))
+                        set_status(p.status, DEV_TIMEOUT_DRAIN);
+                }
+            }
+        }
+    } else if (warp == 1) {
+        // ================= MMA issuer =================
+        if (lane == 0) {
+            constexpr uint32_t idesc = idesc_bf16_f32(BM, BN);
+            int s = 0;
+            uint32_t ph = 0;
+            int it = 0;
+            bool ok = true;
+            for (int t = blockIdx.x; t < total_tiles && ok; t += gridDim.x, ++it) {
+                const int a = it & 1;
+                const uint32_t aph = (it >> 1) & 1;
+                if (!mbar_wait_bounded(&acc_empty[a], aph ^ 1u, s_abort)) {
+                    set_status(p.status, DEV_TIMEOUT_MMA);
+                    *s_abort = 1;
+                    break;
+                }
+                tc_fence_after();
+                const uint32_t d_tmem = tmem_base + a * BN;
+                for (int kb = 0; kb < KB; ++kb) {
+                    if (!mbar_wait_bounded(&full[s], ph, s_abort)) {
+                        set_status(p.status, DEV_TIMEOUT_MMA);
+                        *s_abort = 1;
+                        ok = false;
+                        break;
+                    }
+                    tc_fence_after();
+                    const uint32_t sa = smem_u32(stage_base + s * Geo::STAGE_BYTES);
+                    const uint32_t sb = sa + A_STAGE_BYTES;
+#pragma unroll
+                    for (int kk = 0; kk < BK / 16; ++kk) {
+                        tc_mma_bf16(d_tmem, sdesc_kmajor_sw128(sa + kk * 32),
+                                    sdesc_kmajor_sw128(sb + kk * 32), idesc,
+                                    (kb > 0 || kk > 0) ? 1u : 0u);
+                    }
+                    tc_commit(&empty[s]);
+                    if (++s == STAGES) {
+                        s = 0;
+                        ph ^= 1u;
+                    }
+                }
+                if (ok)
+                    tc_commit(&acc_full[a]);
+            }
+        }
+    } else {
+        // ================= epilogue (warps 2..5) =================
+        const int q = warp & 3;                 // TMEM lane quarter of this warp
+        const int r_in_tile = q * 32 + lane;
+        int it = 0;
+        for (int t = blockIdx.x; t < total_tiles; t += gridDim.x, ++it) {
+            TileInfo ti = tile_info(t, s_prefix, s_off, G, n_tiles, OUTN);
+            const int a = it & 1;
+            const uint32_t aph = (it >> 1) & 1;
+            const bool got = mbar_wait_bounded(&acc_full[a], aph, s_abort);
+            if (!__all_sync(0xffffffffu, got)) {   // tcgen05.ld below needs the whole warp
+                if (lane == 0) {
+                    set_status(p.status, DEV_TIMEOUT_EPILOGUE);
+                    *s_abort = 1;
+                }
+                break;
+            }
+            tc_fence_after();
+            const int64_t row = static_cast<int64_t>(ti.row0) + r_in_tile;
+            const bool row_ok = r_in_tile < ti.rows_valid && row >= 0 && row < p.rows_cap;
+            float scale = 1.0f;
+            if (p.row_scale != nullptr && row_ok)
+                scale = p.row_scale[row];
+            const uint32_t tacc = tmem_base + (static_cast<uint32_t>(q * 32) << 16) + a * BN;
+#pragma unroll 1
+            for (int c = 0; c < OUTN; c += 32) {
+                uint32_t v[32];
+                float o[32];
+                tmem_ld32(tacc + c, v);
+                if (EPI == EPI_SWIGLU) {
+                    uint32_t u[32];
+                    tmem_ld32(tacc + OUTN + c, u);
+                    tmem_wait_ld();
+#pragma unroll
+                    for (int i = 0; i < 32; ++i)
+                        o[i] = silu_f(__uint_as_float(v[i]) * scale) *
+                               (__uint_as_float(u[i]) * scale);
+                } else {
+                    tmem_wait_ld();
+#pragma unroll
+                    for (int i = 0; i < 32; ++i) {
+                        float x = __uint_as_float(v[i]) * scale;
+                        o[i] = (EPI == EPI_RELU) ? fmaxf(x, 0.0f) : x;
+                    }
+                }
+                if (row_ok) {
+                    const int col0 = ti.n0 + c;
+                    if (OUT_F32) {
+                        float *dst = reinterpret_cast<float *>(p.out) + row * p.ld_out + col0;
+                        if (col0 + 32 <= p.n_out) {
+#pragma unroll
+                            for (int i = 0; i < 32; i += 4)
+                                *reinterpret_cast<float4 *>(dst + i) =
+                                    make_float4(o[i], o[i + 1], o[i + 2], o[i + 3]);
+                        } else {
+                            for (int i = 0; i < 32 && col0 + i < p.n_out; ++i)
+                                dst[i] = o[i];
+                        }
+                    } else {
+                        __nv_bfloat16 *dst =
+                            reinterpret_cast<__nv_bfloat16 *>(p.out) + row * p.ld_out + col0;
+                        if (col0 + 32 <= p.n_out) {
+#pragma unroll
+                            for (int i = 0; i < 32; i += 8) {
+                                uint4 w;
+                                w.x = pack_bf16x2(o[i], o[i + 1]);
+                                w.y = pack_bf16x2(o[i + 2], o[i + 3]);
+                                w.z = pack_bf16x2(o[i + 4], o[i + 5]);
+                                w.w = pack_bf16x2(o[i + 6], o[i + 7]);
+                                *reinterpret_cast<uint4 *>(dst + i) = w;
+                            }
+                        } else {
+                            for (int i = 0; i < 32 && col0 + i < p.n_out; ++i)
+                                dst[i] = __float2bfloat16_rn(o[i]);
+                        }
+                    }
+                }
+            }
+            tc_fence_before();
+            mbar_arrive(&acc_empty[a]);
+        }
+    }
+
+    // ---- teardown: MMAs complete, then TMEM is released by its owner warp.
+    // On the normal path the epilogue has already seen the last accumulator
+    // commit (which covers every MMA issued before it).  After an abort, one
+    // more commit on a fresh barrier tells us when the MMAs in flight are done.
+    __syncwarp();
+    if (warp == 1 && lane == 0 && *s_abort) {
+        tc_commit(drain);
+        volatile int never = 0;
+        if (!mbar_wait_bounded(drain, 0, &never))
+            set_status(p.status, DEV_TIMEOUT_DRAIN);
+    }
+    __syncwarp();
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    if (warp == 1)
+        tmem_dealloc(tmem_base, Geo::TMEM_COLS);
+}
+
+// ------------------------------------------------------------------ host
+typedef CUresult (*PFN_encodeTiled)(CUtensorMap *, CUtensorMapDataType, cuuint32_t, void *,
+                                    const cuuint64_t *, const cuuint64_t *, const cuuint32_t *,
+                                    const cuuint32_t *, CUtensorMapInterleave, CUtensorMapSwizzle,
+                                    CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+PFN_encodeTiled get_encode()
+{
+    static PFN_encodeTiled fn = nullptr;
+    static bool tried = false;
+    if (!tried) {
+        tried = true;
+        void *ptr = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &ptr, cudaEnableDefault, &q) ==
+                cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<PFN_encodeTiled>(ptr);
+    }
+    return fn;
+}
+
+// 2-D bf16 tensor map over a [rows, cols] row-major matrix (cols contiguous),
+// box = box_rows x 64 columns, 128-byte swizzle, zero fill out of bounds.
+bool make_map_bf16(CUtensorMap *m, const void *base, int64_t rows, int64_t cols, int box_rows)
+{
+    PFN_encodeTiled enc = get_encode();
+    if (!enc)
+        return false;
+    cuuint64_t dims[2] = {static_cast<cuuint64_t>(cols), static_cast<cuuint64_t>(rows)};
+    cuuint64_t strides[1] = {static_cast<cuuint64_t>(cols) * 2};
+    cuuint32_t box[2] = {static_cast<cuuint32_t>(BK), static_cast<cuuint32_t>(box_rows)};
+    cuuint32_t estr[2] = {1, 1};
+    CUresult r = enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void *>(base), dims,
+                     strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                     CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                     CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    return r == CUDA_SUCCESS;
+}
+
+int sm_count()
+{
+    static int n = 0;
+    if (n == 0) {
+        int dev = 0;
+        cudaGetDevice(&dev);
+        cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev);
+        if (n <= 0)
+            n = 148;
+    }
+    return n;
+}
+
+template <int BN, int EPI, bool OUT_F32>
+cudaError_t launch_impl(const GemmLaunch &L, cudaStream_t stream)
+{
+    using Geo = Geometry<BN, EPI>;
+    CUtensorMap mA, mB, mB2;
+    const int b_box = (EPI == EPI_SWIGLU) ? BN / 2 : BN;
+    if (!make_map_bf16(&mA, L.A, L.a_rows, L.K, BM) ||
+        !make_map_bf16(&mB, L.B, L.b_rows, L.K, b_box))
+        return cudaErrorInvalidValue;
+    if (EPI == EPI_SWIGLU) {
+        if (!make_map_bf16(&mB2, L.B2, L.b_rows, L.K, b_box))
+            return cudaErrorInvalidValue;
+    } else {
+        mB2 = mB;
+    }
+    static bool attr_set = false;
+    if (!attr_set) {
+        cudaError_t e = cudaFuncSetAttribute(grouped_gemm_tc<BN, EPI, OUT_F32>,
+                                             cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                             Geo::SMEM_BYTES);
+        if (e != cudaSuccess)
+            return e;
+        attr_set = true;
+    }
+    GemmParams p;
+    p.offsets = L.offsets;
+    p.rows_single = L.rows_single;
+    p.G = L.G;
+    p.n_out = L.n_out;
+    p.K = L.K;
+    p.out = L.out;
+    p.ld_out = L.ld_out;
+    p.row_scale = L.row_scale;
+    p.rows_cap = L.out_rows;
+    p.status = L.status;
+    const int outn = Geo::OUTN;
+    const int64_t n_tiles = (L.n_out + outn - 1) / outn;
+    const int64_t m_tiles_max = (L.a_rows + BM - 1) / BM + (L.offsets ? L.G : 0);
+    int64_t tiles_max = n_tiles * m_tiles_max;
+    int grid = static_cast<int>(tiles_max < sm_count() ? tiles_max : sm_count());
+    if (grid <= 0)
+        return cudaSuccess;
+    grouped_gemm_tc<BN, EPI, OUT_F32>
+        <<<grid, kThreads, Geo::SMEM_BYTES, stream>>>(mA, mB, mB2, p);
+    count_launches(1);
+    return cudaGetLastError();
+}
+
+}  // namespace
+
+cudaError_t launch_grouped_gemm(const GemmLaunch &L, cudaStream_t stream)
+{
+    if (L.G > kMaxGroups || L.G < 1)
+        return cudaErrorInvalidValue;
+    switch (L.epi) {
+    case EPI_SWIGLU:
+        return launch_impl<256, EPI_SWIGLU, false>(L, stream);
+    case EPI_RELU:
+        return launch_impl<256, EPI_RELU, false>(L, stream);
+    case EPI_STORE:
+    default:
+        if (L.out_f32) {
+            if (L.n_out <= 128)
+                return launch_impl<128, EPI_STORE, true>(L, stream);
+            return launch_impl<256, EPI_STORE, true>(L, stream);
+        }
+        return launch_impl<256, EPI_STORE, false>(L, stream);
+    }
+}
+
+}  // namespace moe

@@ -1,0 +1,103 @@
+// Host-side launchers of the libmoe_b200 kernels (internal interface between
+// the C ABI layer and the kernel files).
+#pragma once
+
+#include <cstdint>
+#include <cuda_runtime.h>
+
+namespace moe {
+
+// Count of kernel launches made by the library (reported by moe_launch_count).
+void count_launches(int n);
+
+enum EpiKind { EPI_STORE = 0, EPI_RELU = 1, EPI_SWIGLU = 2 };
+
+// Grouped GEMM on tcgen05 tensor cores: see gemm_tc.cu.
+struct GemmLaunch {
+    int epi;                 // EpiKind
+    bool out_f32;            // fp32 output (router logits) instead of bf16
+    const void *A;           // [a_rows, K] bf16
+    int64_t a_rows;
+    int32_t K;
+    const void *B;           // [b_rows, K] bf16 (groups stacked: g * n_out + n)
+    const void *B2;          // second weight (W3) for SwiGLU, same shape as B
+    int64_t b_rows;
+    const int32_t *offsets;  // [G+1] device row offsets, or null for one group of rows_single
+    int32_t rows_single;
+    int32_t G;
+    int32_t n_out;
+    void *out;               // [out_rows, ld_out]
+    int64_t out_rows;
+    int64_t ld_out;
+    const float *row_scale;  // [a_rows] or null
+    uint32_t *status;
+};
+cudaError_t launch_grouped_gemm(const GemmLaunch &L, cudaStream_t stream);
+
+// fp32 CUDA-core grouped GEMM (fp32 layers): see ffn_simt.cu.
+cudaError_t launch_simt_gemm_f32(int epi, const float *A, int64_t rows_cap, int32_t K,
+                                 const float *B, const float *B2, int32_t n_out,
+                                 const int32_t *offsets, int32_t G, int32_t rows_single,
+                                 float *out, cudaStream_t stream);
+
+// Router: see router.cu.
+struct RouterLaunch {
+    int dtype;               // MOE_F32 / MOE_BF16
+    const void *x;
+    const void *Wg;
+    const float *bias;
+    int64_t T;
+    int32_t d, N, k;
+    int32_t gate_mode, renormalize;
+    const float *logits_in;  // large-N path: fp32 logits from the tensor-core GEMM
+    float *logits_out;       // optional fp32 logits (small-N path)
+    int32_t *topk_idx;
+    float *topk_w;
+    double *p_part;          // [router_blocks, N] per-block sums of the full softmax
+    int32_t *p_blocks;       // out: number of blocks used (host value, written by launcher)
+    uint32_t *status;
+};
+constexpr int kRouterMaxBlocks = 1184;
+constexpr int kRouterSmallMaxN = 16;
+cudaError_t launch_router_small(RouterLaunch &L, cudaStream_t stream);
+cudaError_t launch_router_select(RouterLaunch &L, cudaStream_t stream);
+// p_mean[e] = sum over blocks of p_part[b][e] / T, summed in block order.
+cudaError_t launch_p_finalize(const double *p_part, int32_t p_blocks, int32_t N, int64_t T,
+                              float *p_mean, cudaStream_t stream);
+
+// Dispatch: see dispatch.cu.
+constexpr int kDispChunk = 2048;      // (token, slot) pairs per block
+struct DispatchLaunch {
+    int dtype;                // element type of x
+    int fp8;                  // quantise rows to E4M3 + per-row scale
+    const void *x;
+    int64_t T;
+    int32_t d, N, k;
+    int64_t capacity;         // -1 = unlimited
+    const int32_t *topk_idx;
+    int32_t *block_base;      // [nblk, N] workspace
+    int32_t *counts;          // [N]
+    int32_t *offsets;         // [N+1]
+    int32_t *perm;            // [T*k]
+    int32_t *inv_row;         // [T*k]
+    uint8_t *drop;            // [T*k]
+    void *x_perm;             // [T*k, d]
+    float *x_scale;           // [T*k] (fp8)
+    void *x_bf16_copy;        // optional [T*k, d] bf16 of the fp8 codes (GEMM operand)
+    const float *p_mean;      // optional in [N] (router output), needed for aux_loss
+    float *f;                 // optional out [N]
+    float *aux_loss;          // optional out [1]
+    float aux_alpha;
+    uint32_t *status;
+};
+cudaError_t launch_dispatch(const DispatchLaunch &L, cudaStream_t stream);
+// E4M3 codes -> bf16 (exact) for rows < offsets[N].
+cudaError_t launch_fp8_to_bf16(const uint8_t *q, int64_t rows_cap, int32_t d,
+                               const int32_t *offsets, int32_t N, void *out, cudaStream_t stream);
+
+// Combine: see combine.cu.
+cudaError_t launch_combine(int dtype, const void *y_perm, const int32_t *inv_row,
+                           const float *topk_w, const void *y_shared, void *y, int64_t T,
+                           int32_t d, int32_t k, uint32_t *status, cudaStream_t stream);
+
+}  // namespace moe

@@ -1,0 +1,589 @@
+// C ABI of libmoe_b200 (declared in include/moe.h): argument validation,
+// workspace layout and the launch sequence of each stage.  No kernel code.
+#include <atomic>
+#include <cstdio>
+#include <cstring>
+#include <mutex>
+#include <vector>
+
+#include "common.cuh"
+#include "kernels.h"
+#include "moe.h"
+
+namespace moe {
+static std::atomic<uint64_t> g_launches{0};
+void count_launches(int n) { g_launches.fetch_add(static_cast<uint64_t>(n)); }
+}  // namespace moe
+
+namespace {
+
+thread_local char g_last_error[256] = "";
+
+// Stage timing of moe_layer_forward (moe_profile_begin / moe_profile_end).
+// Boundary b of a call is recorded before stage b starts; boundary 6 after
+// the combine.  Stages that a call does not run record back-to-back events.
+constexpr int kMarks = MOE_PROFILE_STAGES + 1;
+struct Profiler {
+    std::mutex mu;
+    bool on = false;
+    int max_steps = 0;
+    int steps = 0;
+    std::vector<cudaEvent_t> ev;
+};
+Profiler g_prof;
+
+void prof_mark(int boundary, cudaStream_t s)
+{
+    if (!g_prof.on || g_prof.steps >= g_prof.max_steps)
+        return;
+    cudaEventRecord(g_prof.ev[static_cast<size_t>(g_prof.steps) * kMarks + boundary], s);
+}
+
+moe_status cuda_fail(cudaError_t e)
+{
+    std::snprintf(g_last_error, sizeof(g_last_error), "%s: %s", cudaGetErrorName(e),
+                  cudaGetErrorString(e));
+    return MOE_ERR_CUDA;
+}
+
+#define MOE_CUDA(call)                          \
+    do {                                        \
+        cudaError_t e_ = (call);                \
+        if (e_ != cudaSuccess)                  \
+            return cuda_fail(e_);               \
+    } while (0)
+
+size_t up256(size_t v) { return (v + 255) & ~static_cast<size_t>(255); }
+
+int elem_size(int dt) { return dt == MOE_F32 ? 4 : (dt == MOE_BF16 ? 2 : 1); }
+
+bool aligned(const void *p, size_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
+
+// Offsets of the workspace regions (bytes from the workspace start).
+struct Layout {
+    size_t status, p_part, logits, topk_idx, topk_w, p_mean, counts, offsets, block_base, perm,
+        inv_row, drop, x_scale, x_perm, x_gemm, h, y_perm, hs, ys, total;
+};
+
+bool config_ok(const moe_config *c)
+{
+    if (!c)
+        return false;
+    if (c->T < 0 || c->d <= 0 || c->N < 1 || c->N > 256 || c->k < 1 || c->k > 8 || c->k > c->N ||
+        c->H <= 0 || c->H_shared < 0)
+        return false;
+    if (c->dtype != MOE_F32 && c->dtype != MOE_BF16)
+        return false;
+    if (c->dispatch_dtype != c->dtype &&
+        !(c->dispatch_dtype == MOE_FP8_E4M3 && c->dtype == MOE_BF16))
+        return false;
+    if (c->act != MOE_ACT_RELU && c->act != MOE_ACT_SWIGLU)
+        return false;
+    if (c->gate_mode != MOE_GATE_TOPK_THEN_SOFTMAX && c->gate_mode != MOE_GATE_SOFTMAX_THEN_TOPK)
+        return false;
+    if (c->renormalize != 0 && c->renormalize != 1)
+        return false;
+    const int align = (c->dtype == MOE_BF16) ? 8 : 4;
+    if (c->d % align || c->H % align || c->H_shared % align)
+        return false;
+    if (c->T * c->k > 0x7FFFFFFFll)
+        return false;
+    if (c->dtype == MOE_F32) {
+        // fp32 layers: CUDA-core router (N <= 16) and a row-staged SIMT GEMM
+        if (c->N > moe::kRouterSmallMaxN || c->d > 12288 || c->H > 12288 || c->H_shared > 12288)
+            return false;
+    }
+    return true;
+}
+
+Layout layout_of(const moe_config &c)
+{
+    Layout L{};
+    const size_t T = static_cast<size_t>(c.T), N = c.N, k = c.k, d = c.d, H = c.H;
+    const size_t rows = T * k;
+    const size_t es = elem_size(c.dtype);
+    const size_t nblk = (rows + moe::kDispChunk - 1) / moe::kDispChunk;
+    size_t o = 0;
+    auto take = [&](size_t bytes) {
+        size_t at = o;
+        o += up256(bytes);
+        return at;
+    };
+    L.status = take(256);
+    L.p_part = take(static_cast<size_t>(moe::kRouterMaxBlocks) * N * sizeof(double));
+    L.logits = take(N > static_cast<size_t>(moe::kRouterSmallMaxN) ? T * N * 4 : 0);
+    L.topk_idx = take(rows * 4);
+    L.topk_w = take(rows * 4);
+    L.p_mean = take(N * 4);
+    L.counts = take(N * 4);
+    L.offsets = take((N + 1) * 4);
+    L.block_base = take(nblk * N * 4);
+    L.perm = take(rows * 4);
+    L.inv_row = take(rows * 4);
+    L.drop = take(rows);
+    L.x_scale = take(rows * 4);
+    L.x_perm = take(rows * d * elem_size(c.dispatch_dtype));
+    L.x_gemm = take(c.dispatch_dtype == MOE_FP8_E4M3 ? rows * d * 2 : 0);
+    L.h = take(rows * H * es);
+    L.y_perm = take(rows * d * es);
+    L.hs = take(c.H_shared > 0 ? T * static_cast<size_t>(c.H_shared) * es : 0);
+    L.ys = take(c.H_shared > 0 ? T * d * es : 0);
+    L.total = o;
+    return L;
+}
+
+struct Ws {
+    uint8_t *base;
+    Layout L;
+    template <typename P>
+    P *at(size_t off) const
+    {
+        return reinterpret_cast<P *>(base + off);
+    }
+    uint32_t *status() const { return at<uint32_t>(L.status); }
+};
+
+moe_status check_ws(const moe_config *c, void *ws, size_t ws_bytes, Ws *out)
+{
+    if (!ws || !aligned(ws, 256))
+        return MOE_ERR_WORKSPACE;
+    Layout L = layout_of(*c);
+    if (ws_bytes < L.total)
+        return MOE_ERR_WORKSPACE;
+    out->base = static_cast<uint8_t *>(ws);
+    out->L = L;
+    return MOE_OK;
+}
+
+// ---------------------------------------------------------------- stages
+moe_status run_router(const moe_config &c, const void *x, const void *Wg, const float *bias,
+                      float *logits, int32_t *topk_idx, float *topk_w, float *p_mean,
+                      const Ws &w, cudaStream_t s)
+{
+    if (c.T == 0) {
+        if (p_mean)
+            MOE_CUDA(cudaMemsetAsync(p_mean, 0, c.N * sizeof(float), s));
+        return MOE_OK;
+    }
+    moe::RouterLaunch R{};
+    int32_t blocks = 0;
+    R.dtype = c.dtype;
+    R.x = x;
+    R.Wg = Wg;
+    R.bias = bias;
+    R.T = c.T;
+    R.d = c.d;
+    R.N = c.N;
+    R.k = c.k;
+    R.gate_mode = c.gate_mode;
+    R.renormalize = c.renormalize;
+    R.topk_idx = topk_idx;
+    R.topk_w = topk_w;
+    R.p_part = w.at<double>(w.L.p_part);
+    R.p_blocks = &blocks;
+    R.status = w.status();
+    if (c.N <= moe::kRouterSmallMaxN) {
+        R.logits_out = logits;
+        MOE_CUDA(moe::launch_router_small(R, s));
+    } else {
+        float *lg = logits ? logits : w.at<float>(w.L.logits);
+        moe::GemmLaunch G{};
+        G.epi = moe::EPI_STORE;
+        G.out_f32 = true;
+        G.A = x;
+        G.a_rows = c.T;
+        G.K = c.d;
+        G.B = Wg;
+        G.B2 = nullptr;
+        G.b_rows = c.N;
+        G.offsets = nullptr;
+        G.rows_single = static_cast<int32_t>(c.T);
+        G.G = 1;
+        G.n_out = c.N;
+        G.out = lg;
+        G.out_rows = c.T;
+        G.ld_out = c.N;
+        G.row_scale = nullptr;
+        G.status = w.status();
+        MOE_CUDA(moe::launch_grouped_gemm(G, s));
+        R.logits_in = lg;
+        MOE_CUDA(moe::launch_router_select(R, s));
+    }
+    if (p_mean)
+        MOE_CUDA(moe::launch_p_finalize(R.p_part, blocks, c.N, c.T, p_mean, s));
+    return MOE_OK;
+}
+
+moe_status run_dispatch(const moe_config &c, const void *x, const int32_t *topk_idx,
+                        int32_t *counts, int32_t *offsets, int32_t *perm, int32_t *inv_row,
+                        uint8_t *drop, void *x_perm, float *x_scale, void *x_bf16_copy,
+                        const float *p_mean, float *f, float *aux_loss, const Ws &w,
+                        cudaStream_t s)
+{
+    if (c.T == 0) {
+        MOE_CUDA(cudaMemsetAsync(counts, 0, c.N * sizeof(int32_t), s));
+        MOE_CUDA(cudaMemsetAsync(offsets, 0, (c.N + 1) * sizeof(int32_t), s));
+        if (f)
+            MOE_CUDA(cudaMemsetAsync(f, 0, c.N * sizeof(float), s));
+        if (aux_loss)
+            MOE_CUDA(cudaMemsetAsync(aux_loss, 0, sizeof(float), s));
+        return MOE_OK;
+    }
+    moe::DispatchLaunch D{};
+    D.dtype = c.dtype;
+    D.fp8 = c.dispatch_dtype == MOE_FP8_E4M3;
+    D.x = x;
+    D.T = c.T;
+    D.d = c.d;
+    D.N = c.N;
+    D.k = c.k;
+    D.capacity = -1;
+    if (c.capacity_factor > 0.0f)
+        D.capacity = static_cast<int64_t>(static_cast<double>(c.capacity_factor) *
+                                          static_cast<double>(c.T) / static_cast<double>(c.N));
+    D.topk_idx = topk_idx;
+    D.block_base = w.at<int32_t>(w.L.block_base);
+    D.counts = counts;
+    D.offsets = offsets;
+    D.perm = perm;
+    D.inv_row = inv_row;
+    D.drop = drop;
+    D.x_perm = x_perm;
+    D.x_scale = x_scale;
+    D.x_bf16_copy = x_bf16_copy;
+    D.p_mean = p_mean;
+    D.f = f;
+    D.aux_loss = aux_loss;
+    D.aux_alpha = c.aux_alpha;
+    D.status = w.status();
+    MOE_CUDA(moe::launch_dispatch(D, s));
+    return MOE_OK;
+}
+
+// Dense FFN over grouped rows: up (with activation) into h, down into out.
+moe_status run_ffn(const moe_config &c, const void *A, const float *row_scale, int64_t rows_cap,
+                   const int32_t *offsets, int32_t G, int32_t rows_single, int32_t H,
+                   const void *W1, const void *W3, const void *W2, void *h, void *out,
+                   uint32_t *status, cudaStream_t s, int mark_between = -1)
+{
+    if (rows_cap == 0)
+        return MOE_OK;
+    const int epi = c.act == MOE_ACT_SWIGLU ? moe::EPI_SWIGLU : moe::EPI_RELU;
+    if (c.dtype == MOE_F32) {
+        MOE_CUDA(moe::launch_simt_gemm_f32(epi, static_cast<const float *>(A), rows_cap, c.d,
+                                           static_cast<const float *>(W1),
+                                           static_cast<const float *>(W3), H, offsets, G,
+                                           rows_single, static_cast<float *>(h), s));
+        if (mark_between >= 0)
+            prof_mark(mark_between, s);
+        MOE_CUDA(moe::launch_simt_gemm_f32(moe::EPI_STORE, static_cast<const float *>(h), rows_cap,
+                                           H, static_cast<const float *>(W2), nullptr, c.d,
+                                           offsets, G, rows_single, static_cast<float *>(out), s));
+        return MOE_OK;
+    }
+    moe::GemmLaunch U{};
+    U.epi = epi;
+    U.out_f32 = false;
+    U.A = A;
+    U.a_rows = rows_cap;
+    U.K = c.d;
+    U.B = W1;
+    U.B2 = W3;
+    U.b_rows = static_cast<int64_t>(G) * H;
+    U.offsets = offsets;
+    U.rows_single = rows_single;
+    U.G = G;
+    U.n_out = H;
+    U.out = h;
+    U.out_rows = rows_cap;
+    U.ld_out = H;
+    U.row_scale = row_scale;
+    U.status = status;
+    MOE_CUDA(moe::launch_grouped_gemm(U, s));
+    if (mark_between >= 0)
+        prof_mark(mark_between, s);
+    moe::GemmLaunch Dn{};
+    Dn.epi = moe::EPI_STORE;
+    Dn.out_f32 = false;
+    Dn.A = h;
+    Dn.a_rows = rows_cap;
+    Dn.K = H;
+    Dn.B = W2;
+    Dn.B2 = nullptr;
+    Dn.b_rows = static_cast<int64_t>(G) * c.d;
+    Dn.offsets = offsets;
+    Dn.rows_single = rows_single;
+    Dn.G = G;
+    Dn.n_out = c.d;
+    Dn.out = out;
+    Dn.out_rows = rows_cap;
+    Dn.ld_out = c.d;
+    Dn.row_scale = nullptr;
+    Dn.status = status;
+    MOE_CUDA(moe::launch_grouped_gemm(Dn, s));
+    return MOE_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+size_t moe_workspace_bytes(const moe_config *cfg)
+{
+    if (!config_ok(cfg))
+        return 0;
+    return layout_of(*cfg).total;
+}
+
+moe_status moe_router(const moe_config *cfg, const void *x, const void *Wg, const float *bias,
+                      float *logits, int32_t *topk_idx, float *topk_w, float *p_mean,
+                      void *workspace, size_t workspace_bytes, void *stream)
+{
+    if (!config_ok(cfg))
+        return MOE_ERR_INVALID_ARG;
+    if (cfg->T > 0 && (!x || !Wg || !topk_idx || !topk_w || !aligned(x, 16) || !aligned(Wg, 16)))
+        return MOE_ERR_INVALID_ARG;
+    if (logits && !aligned(logits, 16))
+        return MOE_ERR_INVALID_ARG;
+    Ws w;
+    moe_status st = check_ws(cfg, workspace, workspace_bytes, &w);
+    if (st != MOE_OK)
+        return st;
+    return run_router(*cfg, x, Wg, bias, logits, topk_idx, topk_w, p_mean, w,
+                      static_cast<cudaStream_t>(stream));
+}
+
+moe_status moe_dispatch(const moe_config *cfg, const void *x, const int32_t *topk_idx,
+                        int32_t *expert_counts, int32_t *expert_offsets, int32_t *perm,
+                        int32_t *inv_row, uint8_t *drop_mask, void *x_perm, float *x_scale,
+                        const float *p_mean, float *f, float *aux_loss,
+                        void *workspace, size_t workspace_bytes, void *stream)
+{
+    if (!config_ok(cfg))
+        return MOE_ERR_INVALID_ARG;
+    if (!expert_counts || !expert_offsets)
+        return MOE_ERR_INVALID_ARG;
+    if (cfg->T > 0 && (!x || !topk_idx || !perm || !inv_row || !drop_mask || !x_perm ||
+                       !aligned(x, 16) || !aligned(x_perm, 16)))
+        return MOE_ERR_INVALID_ARG;
+    if (cfg->dispatch_dtype == MOE_FP8_E4M3 && cfg->T > 0 && !x_scale)
+        return MOE_ERR_INVALID_ARG;
+    if (aux_loss && !p_mean)
+        return MOE_ERR_INVALID_ARG;
+    Ws w;
+    moe_status st = check_ws(cfg, workspace, workspace_bytes, &w);
+    if (st != MOE_OK)
+        return st;
+    return run_dispatch(*cfg, x, topk_idx, expert_counts, expert_offsets, perm, inv_row,
+                        drop_mask, x_perm, x_scale, nullptr, p_mean, f, aux_loss, w,
+                        static_cast<cudaStream_t>(stream));
+}
+
+moe_status moe_expert_ffn(const moe_config *cfg, const void *x_perm, const float *x_scale,
+                          const int32_t *expert_offsets, const void *W1, const void *W3,
+                          const void *W2, void *y_perm,
+                          void *workspace, size_t workspace_bytes, void *stream)
+{
+    if (!config_ok(cfg))
+        return MOE_ERR_INVALID_ARG;
+    const bool swiglu = cfg->act == MOE_ACT_SWIGLU;
+    if (cfg->T > 0 && (!x_perm || !expert_offsets || !W1 || !W2 || !y_perm || (swiglu && !W3) ||
+                       !aligned(x_perm, 16) || !aligned(W1, 16) || !aligned(W2, 16) ||
+                       (swiglu && !aligned(W3, 16)) || !aligned(y_perm, 16)))
+        return MOE_ERR_INVALID_ARG;
+    const bool fp8 = cfg->dispatch_dtype == MOE_FP8_E4M3;
+    if (fp8 && cfg->T > 0 && !x_scale)
+        return MOE_ERR_INVALID_ARG;
+    Ws w;
+    moe_status st = check_ws(cfg, workspace, workspace_bytes, &w);
+    if (st != MOE_OK)
+        return st;
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    const int64_t rows_cap = cfg->T * cfg->k;
+    const void *A = x_perm;
+    if (fp8 && rows_cap > 0) {
+        MOE_CUDA(moe::launch_fp8_to_bf16(static_cast<const uint8_t *>(x_perm), rows_cap, cfg->d,
+                                         expert_offsets, cfg->N, w.at<void>(w.L.x_gemm), s));
+        A = w.at<void>(w.L.x_gemm);
+    }
+    return run_ffn(*cfg, A, fp8 ? x_scale : nullptr, rows_cap, expert_offsets, cfg->N, 0, cfg->H,
+                   W1, swiglu ? W3 : nullptr, W2, w.at<void>(w.L.h), y_perm, w.status(), s);
+}
+
+moe_status moe_combine(const moe_config *cfg, const void *y_perm, const int32_t *inv_row,
+                       const float *topk_w, const void *y_shared, void *y,
+                       void *workspace, size_t workspace_bytes, void *stream)
+{
+    if (!config_ok(cfg))
+        return MOE_ERR_INVALID_ARG;
+    if (cfg->T > 0 && (!y_perm || !inv_row || !topk_w || !y || !aligned(y_perm, 16) ||
+                       !aligned(y, 16) || (y_shared && !aligned(y_shared, 16))))
+        return MOE_ERR_INVALID_ARG;
+    Ws w;
+    moe_status st = check_ws(cfg, workspace, workspace_bytes, &w);
+    if (st != MOE_OK)
+        return st;
+    MOE_CUDA(moe::launch_combine(cfg->dtype, y_perm, inv_row, topk_w, y_shared, y, cfg->T, cfg->d,
+                                 cfg->k, w.status(), static_cast<cudaStream_t>(stream)));
+    return MOE_OK;
+}
+
+moe_status moe_layer_forward(const moe_config *cfg, const void *x, const void *Wg,
+                             const float *bias, const void *W1, const void *W3, const void *W2,
+                             const void *Ws1, const void *Ws3, const void *Ws2, void *y,
+                             int32_t *topk_idx, float *topk_w, int32_t *expert_counts,
+                             float *f, float *p_mean, float *aux_loss,
+                             void *workspace, size_t workspace_bytes, void *stream)
+{
+    if (!config_ok(cfg))
+        return MOE_ERR_INVALID_ARG;
+    const moe_config &c = *cfg;
+    const bool swiglu = c.act == MOE_ACT_SWIGLU;
+    const bool shared = c.H_shared > 0;
+    if (c.T > 0) {
+        if (!x || !Wg || !W1 || !W2 || !y || (swiglu && !W3))
+            return MOE_ERR_INVALID_ARG;
+        if (!aligned(x, 16) || !aligned(Wg, 16) || !aligned(W1, 16) || !aligned(W2, 16) ||
+            (swiglu && !aligned(W3, 16)) || !aligned(y, 16))
+            return MOE_ERR_INVALID_ARG;
+        if (shared && (!Ws1 || !Ws2 || (swiglu && !Ws3) || !aligned(Ws1, 16) ||
+                       !aligned(Ws2, 16) || (swiglu && !aligned(Ws3, 16))))
+            return MOE_ERR_INVALID_ARG;
+    }
+    Ws w;
+    moe_status st = check_ws(cfg, workspace, workspace_bytes, &w);
+    if (st != MOE_OK)
+        return st;
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    int32_t *idx = topk_idx ? topk_idx : w.at<int32_t>(w.L.topk_idx);
+    float *gw = topk_w ? topk_w : w.at<float>(w.L.topk_w);
+    int32_t *counts = expert_counts ? expert_counts : w.at<int32_t>(w.L.counts);
+    float *pm = p_mean ? p_mean : ((aux_loss != nullptr) ? w.at<float>(w.L.p_mean) : nullptr);
+    const bool fp8 = c.dispatch_dtype == MOE_FP8_E4M3;
+    int32_t *offsets = w.at<int32_t>(w.L.offsets);
+
+    prof_mark(0, s);
+    st = run_router(c, x, Wg, bias, nullptr, idx, gw, pm, w, s);
+    if (st != MOE_OK)
+        return st;
+    prof_mark(1, s);
+    st = run_dispatch(c, x, idx, counts, offsets, w.at<int32_t>(w.L.perm),
+                      w.at<int32_t>(w.L.inv_row), w.at<uint8_t>(w.L.drop), w.at<void>(w.L.x_perm),
+                      w.at<float>(w.L.x_scale), fp8 ? w.at<void>(w.L.x_gemm) : nullptr, pm, f,
+                      aux_loss, w, s);
+    if (st != MOE_OK)
+        return st;
+    prof_mark(2, s);
+    if (c.T == 0) {
+        for (int b = 3; b < kMarks; ++b)
+            prof_mark(b, s);
+        if (g_prof.on && g_prof.steps < g_prof.max_steps)
+            ++g_prof.steps;
+        return MOE_OK;
+    }
+    const int64_t rows_cap = c.T * c.k;
+    st = run_ffn(c, fp8 ? w.at<void>(w.L.x_gemm) : w.at<void>(w.L.x_perm),
+                 fp8 ? w.at<float>(w.L.x_scale) : nullptr, rows_cap, offsets, c.N, 0, c.H, W1,
+                 swiglu ? W3 : nullptr, W2, w.at<void>(w.L.h), w.at<void>(w.L.y_perm), w.status(),
+                 s, 3);
+    if (st != MOE_OK)
+        return st;
+    prof_mark(4, s);
+    void *ys = nullptr;
+    if (shared) {
+        ys = w.at<void>(w.L.ys);
+        st = run_ffn(c, x, nullptr, c.T, nullptr, 1, static_cast<int32_t>(c.T), c.H_shared, Ws1,
+                     swiglu ? Ws3 : nullptr, Ws2, w.at<void>(w.L.hs), ys, w.status(), s);
+        if (st != MOE_OK)
+            return st;
+    }
+    prof_mark(5, s);
+    MOE_CUDA(moe::launch_combine(c.dtype, w.at<void>(w.L.y_perm), w.at<int32_t>(w.L.inv_row), gw,
+                                 ys, y, c.T, c.d, c.k, w.status(), s));
+    prof_mark(6, s);
+    if (g_prof.on && g_prof.steps < g_prof.max_steps)
+        ++g_prof.steps;
+    return MOE_OK;
+}
+
+moe_status moe_check_status(void *workspace, void *stream, uint32_t *detail)
+{
+    if (!workspace || !aligned(workspace, 256))
+        return MOE_ERR_WORKSPACE;
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    uint32_t word = 0;
+    MOE_CUDA(cudaMemcpyAsync(&word, workspace, sizeof(word), cudaMemcpyDeviceToHost, s));
+    MOE_CUDA(cudaStreamSynchronize(s));
+    if (word != 0) {
+        MOE_CUDA(cudaMemsetAsync(workspace, 0, sizeof(word), s));
+        MOE_CUDA(cudaStreamSynchronize(s));
+    }
+    if (detail)
+        *detail = word;
+    if (word & moe::DEV_TIMEOUT_ANY)
+        return MOE_ERR_TIMEOUT;
+    return word ? MOE_ERR_DEVICE_STATUS : MOE_OK;
+}
+
+const char *moe_status_string(moe_status s)
+{
+    switch (s) {
+    case MOE_OK: return "ok";
+    case MOE_ERR_INVALID_ARG: return "invalid argument";
+    case MOE_ERR_UNSUPPORTED: return "unsupported configuration";
+    case MOE_ERR_WORKSPACE: return "workspace missing, misaligned or too small";
+    case MOE_ERR_CUDA: return "CUDA error";
+    case MOE_ERR_DEVICE_STATUS: return "a kernel recorded an anomaly in the status word";
+    case MOE_ERR_TIMEOUT: return "a bounded device wait gave up";
+    }
+    return "unknown status";
+}
+
+const char *moe_last_error_string(void) { return g_last_error; }
+
+uint64_t moe_launch_count(void) { return moe::g_launches.load(); }
+
+moe_status moe_profile_begin(int max_steps)
+{
+    std::lock_guard<std::mutex> lk(g_prof.mu);
+    if (max_steps <= 0 || g_prof.on)
+        return MOE_ERR_INVALID_ARG;
+    const size_t need = static_cast<size_t>(max_steps) * kMarks;
+    while (g_prof.ev.size() < need) {
+        cudaEvent_t e;
+        MOE_CUDA(cudaEventCreate(&e));
+        g_prof.ev.push_back(e);
+    }
+    g_prof.max_steps = max_steps;
+    g_prof.steps = 0;
+    g_prof.on = true;
+    return MOE_OK;
+}
+
+moe_status moe_profile_end(float *stage_ms, int *steps)
+{
+    std::lock_guard<std::mutex> lk(g_prof.mu);
+    if (!g_prof.on)
+        return MOE_ERR_INVALID_ARG;
+    g_prof.on = false;
+    double acc[MOE_PROFILE_STAGES] = {0};
+    for (int st = 0; st < g_prof.steps; ++st) {
+        MOE_CUDA(cudaEventSynchronize(g_prof.ev[static_cast<size_t>(st) * kMarks + kMarks - 1]));
+        for (int b = 0; b < MOE_PROFILE_STAGES; ++b) {
+            float ms = 0.0f;
+            MOE_CUDA(cudaEventElapsedTime(&ms, g_prof.ev[static_cast<size_t>(st) * kMarks + b],
+                                          g_prof.ev[static_cast<size_t>(st) * kMarks + b + 1]));
+            acc[b] += ms;
+        }
+    }
+    if (stage_ms)
+        for (int b = 0; b < MOE_PROFILE_STAGES; ++b)
+            stage_ms[b] = static_cast<float>(acc[b]);
+    if (steps)
+        *steps = g_prof.steps;
+    return MOE_OK;
+}
+
+const char *moe_version(void) { return "moe_b200 1.0 sm_100a"; }
+
+}  // extern "C"
