@@ -151,7 +151,7 @@ def traffic_from_profile(kernel_key: str, workload_key: str):
 
 
 # ----------------------------------------------------------------- oracle legs
-def oracle_sample(wl, budget_s: float, max_tokens: int = 64):
+def oracle_sample(wl, budget_s: float, max_tokens: int = 4096):
     """Time the CPU oracle on a bounded sample of the workload's tokens.
 
     Routing (router + dispatch) of the sampled tokens and their expert rows and
@@ -183,8 +183,14 @@ def oracle_sample(wl, budget_s: float, max_tokens: int = 64):
     # warm the weight cache outside the timed region (weights are resident, like HBM)
     for e in range(wl.N):
         get_expert(e)
-    pilot = run(np.arange(1))
-    n = int(max(1, min(max_tokens, budget_s / max(pilot, 1e-3))))
+    # grow the sample until it takes a quarter of the budget, then scale to the budget
+    n = 1
+    while True:
+        pilot = run(np.linspace(0, wl.T - 1, n).astype(np.int64))
+        if pilot >= budget_s / 4 or n >= max_tokens:
+            break
+        n *= 2
+    n = int(max(1, min(max_tokens, n * budget_s / max(pilot, 1e-3))))
     toks = np.linspace(0, wl.T - 1, n).astype(np.int64)
     secs = run(toks)
     desc = (f"{n} of {wl.T} tokens (router, top-k, dispatch and expert FFN + combine of their "
@@ -455,7 +461,7 @@ def wl_key(wl):
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=200)
+    ap.add_argument("--steps", type=int, default=400)
     ap.add_argument("--warmup", type=int, default=10)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--workload", choices=list(synth.WORKLOADS), default="mixtral")

@@ -52,62 +52,80 @@ __global__ void __launch_bounds__(kThreads)
             row[j] = __shfl_sync(0xffffffffu, my_row, j);
             g[j] = __shfl_sync(0xffffffffu, my_g, j);
         }
-        for (int c = lane; c < chunks; c += 32) {
-            constexpr int V = BF16 ? 8 : 4;
-            float acc[V];
+        // U chunks per lane per pass, so U loads per row are in flight at once
+        constexpr int U = 4;
+        constexpr int V = BF16 ? 8 : 4;
+        for (int c0 = lane; c0 < chunks; c0 += 32 * U) {
+            float acc[U][V];
 #pragma unroll
-            for (int i = 0; i < V; ++i)
-                acc[i] = 0.0f;
+            for (int u = 0; u < U; ++u)
+#pragma unroll
+                for (int i = 0; i < V; ++i)
+                    acc[u][i] = 0.0f;
 #pragma unroll
             for (int j = 0; j < kMaxK; ++j) {
                 if (j < k && row[j] >= 0) {
+                    const uint4 *src = reinterpret_cast<const uint4 *>(
+                        y_perm + static_cast<int64_t>(row[j]) * d * esz);
+                    uint4 v[U];
+#pragma unroll
+                    for (int u = 0; u < U; ++u) {
+                        const int c = c0 + 32 * u;
+                        v[u] = c < chunks ? __ldg(src + c) : make_uint4(0, 0, 0, 0);
+                    }
+#pragma unroll
+                    for (int u = 0; u < U; ++u) {
+                        const uint32_t w[4] = {v[u].x, v[u].y, v[u].z, v[u].w};
+                        if (BF16) {
+#pragma unroll
+                            for (int i = 0; i < 4; ++i) {
+                                acc[u][2 * i] = fmaf(g[j], __uint_as_float(w[i] << 16), acc[u][2 * i]);
+                                acc[u][2 * i + 1] =
+                                    fmaf(g[j], __uint_as_float(w[i] & 0xFFFF0000u), acc[u][2 * i + 1]);
+                            }
+                        } else {
+#pragma unroll
+                            for (int i = 0; i < 4; ++i)
+                                acc[u][i] = fmaf(g[j], __uint_as_float(w[i]), acc[u][i]);
+                        }
+                    }
+                }
+            }
+#pragma unroll
+            for (int u = 0; u < U; ++u) {
+                const int c = c0 + 32 * u;
+                if (c >= chunks)
+                    continue;
+                if (y_shared != nullptr) {
                     const uint4 v = __ldg(reinterpret_cast<const uint4 *>(
-                                              y_perm + static_cast<int64_t>(row[j]) * d * esz) +
-                                          c);
+                                              y_shared + t * static_cast<int64_t>(d) * esz) + c);
                     const uint32_t w[4] = {v.x, v.y, v.z, v.w};
                     if (BF16) {
 #pragma unroll
                         for (int i = 0; i < 4; ++i) {
-                            acc[2 * i] = fmaf(g[j], __uint_as_float(w[i] << 16), acc[2 * i]);
-                            acc[2 * i + 1] =
-                                fmaf(g[j], __uint_as_float(w[i] & 0xFFFF0000u), acc[2 * i + 1]);
+                            acc[u][2 * i] += __uint_as_float(w[i] << 16);
+                            acc[u][2 * i + 1] += __uint_as_float(w[i] & 0xFFFF0000u);
                         }
                     } else {
 #pragma unroll
                         for (int i = 0; i < 4; ++i)
-                            acc[i] = fmaf(g[j], __uint_as_float(w[i]), acc[i]);
+                            acc[u][i] += __uint_as_float(w[i]);
                     }
                 }
-            }
-            if (y_shared != nullptr) {
-                const uint4 v = __ldg(
-                    reinterpret_cast<const uint4 *>(y_shared + t * static_cast<int64_t>(d) * esz) + c);
-                const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+                uint4 o;
                 if (BF16) {
-#pragma unroll
-                    for (int i = 0; i < 4; ++i) {
-                        acc[2 * i] += __uint_as_float(w[i] << 16);
-                        acc[2 * i + 1] += __uint_as_float(w[i] & 0xFFFF0000u);
-                    }
+                    o.x = pack_bf16x2(acc[u][0], acc[u][1]);
+                    o.y = pack_bf16x2(acc[u][2], acc[u][3]);
+                    o.z = pack_bf16x2(acc[u][4], acc[u][5]);
+                    o.w = pack_bf16x2(acc[u][6], acc[u][7]);
                 } else {
-#pragma unroll
-                    for (int i = 0; i < 4; ++i)
-                        acc[i] += __uint_as_float(w[i]);
+                    o.x = __float_as_uint(acc[u][0]);
+                    o.y = __float_as_uint(acc[u][1]);
+                    o.z = __float_as_uint(acc[u][2]);
+                    o.w = __float_as_uint(acc[u][3]);
                 }
+                reinterpret_cast<uint4 *>(y + t * static_cast<int64_t>(d) * esz)[c] = o;
             }
-            uint4 o;
-            if (BF16) {
-                o.x = pack_bf16x2(acc[0], acc[1]);
-                o.y = pack_bf16x2(acc[2], acc[3]);
-                o.z = pack_bf16x2(acc[4], acc[5]);
-                o.w = pack_bf16x2(acc[6], acc[7]);
-            } else {
-                o.x = __float_as_uint(acc[0]);
-                o.y = __float_as_uint(acc[1]);
-                o.z = __float_as_uint(acc[2]);
-                o.w = __float_as_uint(acc[3]);
-            }
-            reinterpret_cast<uint4 *>(y + t * static_cast<int64_t>(d) * esz)[c] = o;
         }
     }
 }

@@ -224,8 +224,18 @@ __global__ void __launch_bounds__(kThreads)
         const uint4 *src = reinterpret_cast<const uint4 *>(x + t * static_cast<int64_t>(d) * esz);
         if (!FP8) {
             uint4 *dst = reinterpret_cast<uint4 *>(x_perm + r * static_cast<int64_t>(d) * esz);
-            for (int c = lane; c < chunks; c += 32)
-                dst[c] = __ldg(src + c);
+            constexpr int U = 4;  // loads in flight per lane
+            for (int c0 = lane; c0 < chunks; c0 += 32 * U) {
+                uint4 v[U];
+#pragma unroll
+                for (int u = 0; u < U; ++u)
+                    if (c0 + 32 * u < chunks)
+                        v[u] = __ldg(src + c0 + 32 * u);
+#pragma unroll
+                for (int u = 0; u < U; ++u)
+                    if (c0 + 32 * u < chunks)
+                        dst[c0 + 32 * u] = v[u];
+            }
         } else {
             float amax = 0.0f;
             for (int c = lane; c < chunks; c += 32) {

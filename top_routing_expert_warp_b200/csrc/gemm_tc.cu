@@ -52,6 +52,7 @@ struct GemmParams {
     int64_t ld_out;          // elements
     const float *row_scale;  // multiply each accumulator row by row_scale[r], or null
     int64_t rows_cap;        // rows allocated in out (and row_scale); rows beyond are never written
+    int32_t prefetch;        // 1: prefetch weight boxes into L2 ahead of their loads
     uint32_t *status;
 };
 
@@ -67,8 +68,19 @@ struct Geometry {
     static constexpr int SMEM_BYTES = 1024 + STAGES * STAGE_BYTES + AUX_BYTES;
 };
 
+// A partial tile of at most kSwapMaxRows rows runs "swapped": the weight rows
+// are the MMA's M (128 per MMA) and the tile's rows, rounded up to a multiple
+// of 16, its N, so the tensor cores do not pad the rows to 128.
+constexpr int kSwapMaxRows = 112;
+
+// Weight boxes may be prefetched into L2 this many k-blocks before their load
+// (GemmParams::prefetch; helps weight streaming when few CTAs share a tile).
+constexpr int kPrefetchAhead = 8;
+
 struct TileInfo {
     int32_t g, row0, rows_valid, n0;
+    bool swap;
+    int32_t ntok;   // swapped tiles: MMA N (rows_valid rounded up to 16)
 };
 
 // Locate tile t: prefix[g] <= t < prefix[g+1].
@@ -95,6 +107,8 @@ __device__ __forceinline__ TileInfo tile_info(int t, const int32_t *s_prefix,
     ti.row0 = s_off[g] + m_tile * BM;
     ti.rows_valid = min(BM, rows_g - m_tile * BM);
     ti.n0 = n_tile * outn;
+    ti.swap = ti.rows_valid <= kSwapMaxRows;
+    ti.ntok = (ti.rows_valid + 15) & ~15;
     (void)n_tiles;
     return ti;
 }
@@ -104,14 +118,63 @@ __device__ __forceinline__ float silu_f(float a)
     return a / (1.0f + __expf(-a));
 }
 
+// 32 consecutive outputs of one row (columns col0 .. col0+31, masked at n_out).
+template <bool OUT_F32>
+__device__ __forceinline__ void store_row32(void *out, int64_t row_off, int col0, int n_out,
+                                            const float (&o)[32])
+{
+    if (OUT_F32) {
+        float *dst = reinterpret_cast<float *>(out) + row_off + col0;
+        if (col0 + 32 <= n_out) {
+#pragma unroll
+            for (int i = 0; i < 32; i += 4)
+                *reinterpret_cast<float4 *>(dst + i) = make_float4(o[i], o[i + 1], o[i + 2], o[i + 3]);
+        } else {
+#pragma unroll
+            for (int i = 0; i < 32; ++i)
+                if (col0 + i < n_out)
+                    dst[i] = o[i];
+        }
+    } else {
+        __nv_bfloat16 *dst = reinterpret_cast<__nv_bfloat16 *>(out) + row_off + col0;
+        if (col0 + 32 <= n_out) {
+#pragma unroll
+            for (int i = 0; i < 32; i += 8) {
+                uint4 w;
+                w.x = pack_bf16x2(o[i], o[i + 1]);
+                w.y = pack_bf16x2(o[i + 2], o[i + 3]);
+                w.z = pack_bf16x2(o[i + 4], o[i + 5]);
+                w.w = pack_bf16x2(o[i + 6], o[i + 7]);
+                *reinterpret_cast<uint4 *>(dst + i) = w;
+            }
+        } else {
+#pragma unroll
+            for (int i = 0; i < 32; ++i)
+                if (col0 + i < n_out)
+                    dst[i] = __float2bfloat16_rn(o[i]);
+        }
+    }
+}
+
+template <bool OUT_F32>
+__device__ __forceinline__ void store_one(void *out, int64_t off, float v)
+{
+    if (OUT_F32)
+        reinterpret_cast<float *>(out)[off] = v;
+    else
+        reinterpret_cast<__nv_bfloat16 *>(out)[off] = __float2bfloat16_rn(v);
+}
+
 template <int BN, int EPI, bool OUT_F32>
 __global__ void __launch_bounds__(kThreads, 1)
-    grouped_gemm_tc(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
-                    const __grid_constant__ CUtensorMap tmB2, GemmParams p)
+    grouped_gemm_tc(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmA16,
+                    const __grid_constant__ CUtensorMap tmB, const __grid_constant__ CUtensorMap tmB2,
+                    GemmParams p)
 {
     using Geo = Geometry<BN, EPI>;
     constexpr int STAGES = Geo::STAGES;
     constexpr int OUTN = Geo::OUTN;
+    constexpr int HALVES = BN / 128;   // swapped tiles: one M=128 MMA per 128 weight rows
 
     extern __shared__ uint8_t smem_raw[];
     uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
@@ -134,7 +197,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int n_tiles = (p.n_out + OUTN - 1) / OUTN;
     const int KB = (p.K + BK - 1) / BK;
 
-    // ---- group table and tile prefix (warp 2), barriers (warp 0), TMEM (warp 1)
+    // ---- barriers (warp 0), TMEM (warp 1), group table and tile prefix (warp 2)
     if (warp == 0 && lane == 0) {
         for (int s = 0; s < STAGES; ++s) {
             mbar_init(&full[s], 1);
@@ -148,6 +211,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         *s_abort = 0;
         fence_barrier_init();
         tma_prefetch_desc(&tmA);
+        tma_prefetch_desc(&tmA16);
         tma_prefetch_desc(&tmB);
         if (EPI == EPI_SWIGLU)
             tma_prefetch_desc(&tmB2);
@@ -157,7 +221,6 @@ __global__ void __launch_bounds__(kThreads, 1)
         tmem_relinquish();
     }
     if (warp == 2) {
-        // offsets -> smem; per-group tile counts -> inclusive scan over groups
         const int per = (G + 32) / 32;  // G+1 entries of offsets
         for (int i = lane; i <= G; i += 32)
             s_off[i] = p.offsets ? p.offsets[i] : (i == 0 ? 0 : p.rows_single);
@@ -201,12 +264,39 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (lane == 0) {
             int s = 0;
             uint32_t ph = 0;
-            uint32_t last_par[STAGES];
+            uint32_t last_par = 0;  // bit s: parity of the last load issued to stage s
             uint32_t used = 0;
             bool ok = true;
+            // L2 prefetch cursor: kPrefetchAhead k-blocks ahead of the loads in
+            // this CTA's own (tile, k-block) sequence, weights only
+            int pf_t = blockIdx.x, pf_kb = 0, pf_brow = 0;
+            if (pf_t < total_tiles) {
+                const TileInfo pi = tile_info(pf_t, s_prefix, s_off, G, n_tiles, OUTN);
+                pf_brow = pi.g * p.n_out + pi.n0;
+            }
+            auto prefetch_next = [&]() {
+                if (!p.prefetch || pf_t >= total_tiles)
+                    return;
+                tma_prefetch_l2_2d(&tmB, pf_kb * BK, pf_brow);
+                if (EPI == EPI_SWIGLU)
+                    tma_prefetch_l2_2d(&tmB2, pf_kb * BK, pf_brow);
+                if (++pf_kb == KB) {
+                    pf_kb = 0;
+                    pf_t += gridDim.x;
+                    if (pf_t < total_tiles) {
+                        const TileInfo pi = tile_info(pf_t, s_prefix, s_off, G, n_tiles, OUTN);
+                        pf_brow = pi.g * p.n_out + pi.n0;
+                    }
+                }
+            };
+            for (int i = 0; i < kPrefetchAhead; ++i)
+                prefetch_next();
             for (int t = blockIdx.x; t < total_tiles && ok; t += gridDim.x) {
-                TileInfo ti = tile_info(t, s_prefix, s_off, G, n_tiles, OUTN);
+                const TileInfo ti = tile_info(t, s_prefix, s_off, G, n_tiles, OUTN);
                 const int brow = ti.g * p.n_out + ti.n0;
+                const int a_boxes = ti.ntok / 16;          // swapped tile: 16-row boxes
+                const uint32_t bytes = ti.swap ? (a_boxes * 16 * BK * 2 + Geo::B_STAGE_BYTES)
+                                               : Geo::STAGE_BYTES;
                 for (int kb = 0; kb < KB; ++kb) {
                     if (!mbar_wait_bounded(&empty[s], ph ^ 1u, s_abort)) {
                         set_status(p.status, DEV_TIMEOUT_PRODUCER);
@@ -216,15 +306,22 @@ __global__ void __launch_bounds__(kThreads, 1)
                     }
                     uint8_t *sa = stage_base + s * Geo::STAGE_BYTES;
                     uint8_t *sb = sa + A_STAGE_BYTES;
-                    mbar_arrive_expect_tx(&full[s], Geo::STAGE_BYTES);
-                    tma_load_2d(sa, &tmA, &full[s], kb * BK, ti.row0);
+                    mbar_arrive_expect_tx(&full[s], bytes);
+                    if (ti.swap) {
+                        for (int b = 0; b < a_boxes; ++b)
+                            tma_load_2d(sa + b * 16 * BK * 2, &tmA16, &full[s], kb * BK,
+                                        ti.row0 + 16 * b);
+                    } else {
+                        tma_load_2d(sa, &tmA, &full[s], kb * BK, ti.row0);
+                    }
                     if (EPI == EPI_SWIGLU) {
                         tma_load_2d(sb, &tmB, &full[s], kb * BK, brow);
                         tma_load_2d(sb + (BN / 2) * BK * 2, &tmB2, &full[s], kb * BK, brow);
                     } else {
                         tma_load_2d(sb, &tmB, &full[s], kb * BK, brow);
                     }
-                    last_par[s] = ph;
+                    prefetch_next();
+                    last_par = (last_par & ~(1u << s)) | (ph << s);
                     used |= 1u << s;
                     if (++s == STAGES) {
                         s = 0;
@@ -236,7 +333,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             for (int i = 0; i < STAGES; ++i) {
                 if ((used >> i) & 1u) {
                     volatile int never = 0;
-                    if (!mbar_wait_bounded(&full[i], last_par[i], &never))
+                    if (!mbar_wait_bounded(&full[i], (last_par >> i) & 1u, &never))
                         set_status(p.status, DEV_TIMEOUT_DRAIN);
                 }
             }
@@ -244,12 +341,14 @@ __global__ void __launch_bounds__(kThreads, 1)
     } else if (warp == 1) {
         // ================= MMA issuer =================
         if (lane == 0) {
-            constexpr uint32_t idesc = idesc_bf16_f32(BM, BN);
+            constexpr uint32_t idesc_n = idesc_bf16_f32(BM, BN);
             int s = 0;
             uint32_t ph = 0;
             int it = 0;
             bool ok = true;
             for (int t = blockIdx.x; t < total_tiles && ok; t += gridDim.x, ++it) {
+                const TileInfo ti = tile_info(t, s_prefix, s_off, G, n_tiles, OUTN);
+                const uint32_t idesc_s = idesc_bf16_f32(128, ti.ntok);
                 const int a = it & 1;
                 const uint32_t aph = (it >> 1) & 1;
                 if (!mbar_wait_bounded(&acc_empty[a], aph ^ 1u, s_abort)) {
@@ -269,11 +368,22 @@ __global__ void __launch_bounds__(kThreads, 1)
                     tc_fence_after();
                     const uint32_t sa = smem_u32(stage_base + s * Geo::STAGE_BYTES);
                     const uint32_t sb = sa + A_STAGE_BYTES;
+                    if (!ti.swap) {
 #pragma unroll
-                    for (int kk = 0; kk < BK / 16; ++kk) {
-                        tc_mma_bf16(d_tmem, sdesc_kmajor_sw128(sa + kk * 32),
-                                    sdesc_kmajor_sw128(sb + kk * 32), idesc,
-                                    (kb > 0 || kk > 0) ? 1u : 0u);
+                        for (int kk = 0; kk < BK / 16; ++kk)
+                            tc_mma_bf16(d_tmem, sdesc_kmajor_sw128(sa + kk * 32),
+                                        sdesc_kmajor_sw128(sb + kk * 32), idesc_n,
+                                        (kb > 0 || kk > 0) ? 1u : 0u);
+                    } else {
+                        // D^T: weight rows are the MMA's M, the tile's tokens its N
+#pragma unroll
+                        for (int kk = 0; kk < BK / 16; ++kk)
+#pragma unroll
+                            for (int h = 0; h < HALVES; ++h)
+                                tc_mma_bf16(d_tmem + h * 128,
+                                            sdesc_kmajor_sw128(sb + h * 128 * BK * 2 + kk * 32),
+                                            sdesc_kmajor_sw128(sa + kk * 32), idesc_s,
+                                            (kb > 0 || kk > 0) ? 1u : 0u);
                     }
                     tc_commit(&empty[s]);
                     if (++s == STAGES) {
@@ -291,7 +401,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         const int r_in_tile = q * 32 + lane;
         int it = 0;
         for (int t = blockIdx.x; t < total_tiles; t += gridDim.x, ++it) {
-            TileInfo ti = tile_info(t, s_prefix, s_off, G, n_tiles, OUTN);
+            const TileInfo ti = tile_info(t, s_prefix, s_off, G, n_tiles, OUTN);
             const int a = it & 1;
             const uint32_t aph = (it >> 1) & 1;
             const bool got = mbar_wait_bounded(&acc_full[a], aph, s_abort);
@@ -303,62 +413,79 @@ __global__ void __launch_bounds__(kThreads, 1)
                 break;
             }
             tc_fence_after();
-            const int64_t row = static_cast<int64_t>(ti.row0) + r_in_tile;
-            const bool row_ok = r_in_tile < ti.rows_valid && row >= 0 && row < p.rows_cap;
-            float scale = 1.0f;
-            if (p.row_scale != nullptr && row_ok)
-                scale = p.row_scale[row];
             const uint32_t tacc = tmem_base + (static_cast<uint32_t>(q * 32) << 16) + a * BN;
+            if (!ti.swap) {
+                // lane = output row, columns = output features
+                const int64_t row = static_cast<int64_t>(ti.row0) + r_in_tile;
+                const bool row_ok = r_in_tile < ti.rows_valid && row >= 0 && row < p.rows_cap;
+                float scale = 1.0f;
+                if (p.row_scale != nullptr && row_ok)
+                    scale = p.row_scale[row];
 #pragma unroll 1
-            for (int c = 0; c < OUTN; c += 32) {
-                uint32_t v[32];
-                float o[32];
-                tmem_ld32(tacc + c, v);
-                if (EPI == EPI_SWIGLU) {
-                    uint32_t u[32];
-                    tmem_ld32(tacc + OUTN + c, u);
-                    tmem_wait_ld();
+                for (int c = 0; c < OUTN; c += 32) {
+                    uint32_t v[32];
+                    float o[32];
+                    tmem_ld32(tacc + c, v);
+                    if (EPI == EPI_SWIGLU) {
+                        uint32_t u[32];
+                        tmem_ld32(tacc + OUTN + c, u);
+                        tmem_wait_ld();
 #pragma unroll
-                    for (int i = 0; i < 32; ++i)
-                        o[i] = silu_f(__uint_as_float(v[i]) * scale) *
-                               (__uint_as_float(u[i]) * scale);
-                } else {
-                    tmem_wait_ld();
+                        for (int i = 0; i < 32; ++i)
+                            o[i] = silu_f(__uint_as_float(v[i]) * scale) *
+                                   (__uint_as_float(u[i]) * scale);
+                    } else {
+                        tmem_wait_ld();
 #pragma unroll
-                    for (int i = 0; i < 32; ++i) {
-                        float x = __uint_as_float(v[i]) * scale;
-                        o[i] = (EPI == EPI_RELU) ? fmaxf(x, 0.0f) : x;
+                        for (int i = 0; i < 32; ++i) {
+                            float x = __uint_as_float(v[i]) * scale;
+                            o[i] = (EPI == EPI_RELU) ? fmaxf(x, 0.0f) : x;
+                        }
                     }
+                    if (row_ok)
+                        store_row32<OUT_F32>(p.out, row * p.ld_out, ti.n0 + c, p.n_out, o);
                 }
-                if (row_ok) {
-                    const int col0 = ti.n0 + c;
-                    if (OUT_F32) {
-                        float *dst = reinterpret_cast<float *>(p.out) + row * p.ld_out + col0;
-                        if (col0 + 32 <= p.n_out) {
+            } else {
+                // swapped tile: lane = output feature, columns = tokens
+#pragma unroll 1
+                for (int c = 0; c < ti.ntok; c += 16) {
+                    float sc[16];
 #pragma unroll
-                            for (int i = 0; i < 32; i += 4)
-                                *reinterpret_cast<float4 *>(dst + i) =
-                                    make_float4(o[i], o[i + 1], o[i + 2], o[i + 3]);
-                        } else {
-                            for (int i = 0; i < 32 && col0 + i < p.n_out; ++i)
-                                dst[i] = o[i];
+                    for (int i = 0; i < 16; ++i) {
+                        const int64_t row = static_cast<int64_t>(ti.row0) + c + i;
+                        sc[i] = (p.row_scale != nullptr && c + i < ti.rows_valid && row < p.rows_cap)
+                                    ? p.row_scale[row] : 1.0f;
+                    }
+                    if (EPI == EPI_SWIGLU) {
+                        uint32_t v[16], u[16];
+                        tmem_ld16(tacc + c, v);
+                        tmem_ld16(tacc + 128 + c, u);
+                        tmem_wait_ld();
+                        const int col = ti.n0 + r_in_tile;
+#pragma unroll
+                        for (int i = 0; i < 16; ++i) {
+                            const int64_t row = static_cast<int64_t>(ti.row0) + c + i;
+                            const float o = silu_f(__uint_as_float(v[i]) * sc[i]) *
+                                            (__uint_as_float(u[i]) * sc[i]);
+                            if (c + i < ti.rows_valid && row < p.rows_cap && col < p.n_out)
+                                store_one<OUT_F32>(p.out, row * p.ld_out + col, o);
                         }
                     } else {
-                        __nv_bfloat16 *dst =
-                            reinterpret_cast<__nv_bfloat16 *>(p.out) + row * p.ld_out + col0;
-                        if (col0 + 32 <= p.n_out) {
 #pragma unroll
-                            for (int i = 0; i < 32; i += 8) {
-                                uint4 w;
-                                w.x = pack_bf16x2(o[i], o[i + 1]);
-                                w.y = pack_bf16x2(o[i + 2], o[i + 3]);
-                                w.z = pack_bf16x2(o[i + 4], o[i + 5]);
-                                w.w = pack_bf16x2(o[i + 6], o[i + 7]);
-                                *reinterpret_cast<uint4 *>(dst + i) = w;
+                        for (int h = 0; h < HALVES; ++h) {
+                            uint32_t v[16];
+                            tmem_ld16(tacc + h * 128 + c, v);
+                            tmem_wait_ld();
+                            const int col = ti.n0 + h * 128 + r_in_tile;
+#pragma unroll
+                            for (int i = 0; i < 16; ++i) {
+                                const int64_t row = static_cast<int64_t>(ti.row0) + c + i;
+                                float x = __uint_as_float(v[i]) * sc[i];
+                                if (EPI == EPI_RELU)
+                                    x = fmaxf(x, 0.0f);
+                                if (c + i < ti.rows_valid && row < p.rows_cap && col < p.n_out)
+                                    store_one<OUT_F32>(p.out, row * p.ld_out + col, x);
                             }
-                        } else {
-                            for (int i = 0; i < 32 && col0 + i < p.n_out; ++i)
-                                dst[i] = __float2bfloat16_rn(o[i]);
                         }
                     }
                 }
@@ -444,9 +571,10 @@ template <int BN, int EPI, bool OUT_F32>
 cudaError_t launch_impl(const GemmLaunch &L, cudaStream_t stream)
 {
     using Geo = Geometry<BN, EPI>;
-    CUtensorMap mA, mB, mB2;
+    CUtensorMap mA, mA16, mB, mB2;
     const int b_box = (EPI == EPI_SWIGLU) ? BN / 2 : BN;
     if (!make_map_bf16(&mA, L.A, L.a_rows, L.K, BM) ||
+        !make_map_bf16(&mA16, L.A, L.a_rows, L.K, 16) ||
         !make_map_bf16(&mB, L.B, L.b_rows, L.K, b_box))
         return cudaErrorInvalidValue;
     if (EPI == EPI_SWIGLU) {
@@ -474,6 +602,7 @@ cudaError_t launch_impl(const GemmLaunch &L, cudaStream_t stream)
     p.ld_out = L.ld_out;
     p.row_scale = L.row_scale;
     p.rows_cap = L.out_rows;
+    p.prefetch = L.prefetch;
     p.status = L.status;
     const int outn = Geo::OUTN;
     const int64_t n_tiles = (L.n_out + outn - 1) / outn;
@@ -483,7 +612,7 @@ cudaError_t launch_impl(const GemmLaunch &L, cudaStream_t stream)
     if (grid <= 0)
         return cudaSuccess;
     grouped_gemm_tc<BN, EPI, OUT_F32>
-        <<<grid, kThreads, Geo::SMEM_BYTES, stream>>>(mA, mB, mB2, p);
+        <<<grid, kThreads, Geo::SMEM_BYTES, stream>>>(mA, mA16, mB, mB2, p);
     count_launches(1);
     return cudaGetLastError();
 }

@@ -30,6 +30,7 @@ struct GemmLaunch {
     int64_t out_rows;
     int64_t ld_out;
     const float *row_scale;  // [a_rows] or null
+    int32_t prefetch;        // prefetch weight boxes into L2 ahead of their loads
     uint32_t *status;
 };
 cudaError_t launch_grouped_gemm(const GemmLaunch &L, cudaStream_t stream);

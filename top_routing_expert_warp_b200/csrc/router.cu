@@ -16,7 +16,7 @@
 // and all of d), the work here is spread over a warp per token with 16-byte
 // loads, and routing decisions are taken on fp64 logits:
 //   - small N (<= 16): router_small computes every logit with exact products
-//     and fp64 accumulation, then selects;
+//     and compensated accumulation (fp64-level accuracy), then selects;
 //   - large N: the logits come from the tcgen05 GEMM (fp32 accumulation);
 //     router_select takes the best few candidates on those, recomputes the
 //     candidates in fp64 and decides among them, so near-ties are resolved as
@@ -43,28 +43,67 @@ __device__ __forceinline__ double warp_sum(double v)
     return v;
 }
 
-// fp64 dot of 16-byte chunks: bf16 (8 values) or fp32 (4 values); each
-// product is exact in fp64.
+// Accumulator of a dot product: a compensated fp32 pair (hi + lo) for bf16
+// operands, whose products are exact in fp32 (8-bit significands); plain fp64
+// for fp32 operands.  Each 16-byte chunk (8 bf16 products) is summed in fp32,
+// then added to (hi, lo) with Knuth's branch-free TwoSum, so no rounding
+// error accumulates across chunks and the result is as accurate as an fp64
+// sum of the chunk sums, without fp64 or conversion instructions in the loop.
+struct DotAcc {
+    float hi = 0.0f, lo = 0.0f;
+    double d = 0.0;
+    __device__ __forceinline__ void add_chunk_sum(float s)
+    {
+        const float t = hi + s;
+        const float bp = t - hi;
+        lo += (hi - (t - bp)) + (s - bp);
+        hi = t;
+    }
+    __device__ __forceinline__ double value(bool bf16) const
+    {
+        return bf16 ? static_cast<double>(hi) + static_cast<double>(lo) : d;
+    }
+};
+
 template <bool BF16>
-__device__ __forceinline__ double chunk_dot(const uint4 a, const uint4 b, double acc)
+__device__ __forceinline__ void chunk_dot(const float (&xf)[8], const uint4 b, DotAcc &acc)
 {
-    const uint32_t av[4] = {a.x, a.y, a.z, a.w};
     const uint32_t bv[4] = {b.x, b.y, b.z, b.w};
     if (BF16) {
+        float s = xf[0] * __uint_as_float(bv[0] << 16);
+        s = fmaf(xf[1], __uint_as_float(bv[0] & 0xFFFF0000u), s);
 #pragma unroll
-        for (int i = 0; i < 4; ++i) {
-            acc = fma(static_cast<double>(__uint_as_float(av[i] << 16)),
-                      static_cast<double>(__uint_as_float(bv[i] << 16)), acc);
-            acc = fma(static_cast<double>(__uint_as_float(av[i] & 0xFFFF0000u)),
-                      static_cast<double>(__uint_as_float(bv[i] & 0xFFFF0000u)), acc);
+        for (int i = 1; i < 4; ++i) {
+            s = fmaf(xf[2 * i], __uint_as_float(bv[i] << 16), s);
+            s = fmaf(xf[2 * i + 1], __uint_as_float(bv[i] & 0xFFFF0000u), s);
         }
+        acc.add_chunk_sum(s);
     } else {
 #pragma unroll
         for (int i = 0; i < 4; ++i)
-            acc = fma(static_cast<double>(__uint_as_float(av[i])),
-                      static_cast<double>(__uint_as_float(bv[i])), acc);
+            acc.d = fma(static_cast<double>(xf[i]), static_cast<double>(__uint_as_float(bv[i])),
+                        acc.d);
     }
-    return acc;
+}
+
+// The 8 (bf16) or 4 (fp32) values of a 16-byte chunk as floats.
+template <bool BF16>
+__device__ __forceinline__ void unpack_chunk(const uint4 a, float (&xf)[8])
+{
+    const uint32_t av[4] = {a.x, a.y, a.z, a.w};
+    if (BF16) {
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+            xf[2 * i] = __uint_as_float(av[i] << 16);
+            xf[2 * i + 1] = __uint_as_float(av[i] & 0xFFFF0000u);
+        }
+    } else {
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+            xf[i] = __uint_as_float(av[i]);
+            xf[4 + i] = 0.0f;
+        }
+    }
 }
 
 template <bool BF16, int NMAX>
@@ -82,33 +121,30 @@ __global__ void __launch_bounds__(kThreads)
     const uint8_t *x = static_cast<const uint8_t *>(xv);
     const uint8_t *w = static_cast<const uint8_t *>(wv);
 
-    double psum[NMAX];
-#pragma unroll
-    for (int e = 0; e < NMAX; ++e)
-        psum[e] = 0.0;
+    double my_psum = 0.0;  // lane e: this warp's sum of p_e over its tokens
 
     for (int64_t t = static_cast<int64_t>(blockIdx.x) * kWarps + warp; t < T;
          t += static_cast<int64_t>(gridDim.x) * kWarps) {
-        double acc[NMAX];
-#pragma unroll
-        for (int e = 0; e < NMAX; ++e)
-            acc[e] = 0.0;
+        DotAcc da[NMAX];
         const uint4 *xr = reinterpret_cast<const uint4 *>(x + t * static_cast<int64_t>(d) * esz);
+#pragma unroll 2
         for (int c = lane; c < chunks; c += 32) {
-            const uint4 xa = __ldg(xr + c);
+            float xf[8];
+            unpack_chunk<BF16>(__ldg(xr + c), xf);
 #pragma unroll
             for (int e = 0; e < NMAX; ++e) {
                 if (e < N) {
                     const uint4 wa = __ldg(reinterpret_cast<const uint4 *>(
                                                w + static_cast<int64_t>(e) * d * esz) +
                                            c);
-                    acc[e] = chunk_dot<BF16>(xa, wa, acc[e]);
+                    chunk_dot<BF16>(xf, wa, da[e]);
                 }
             }
         }
+        double acc[NMAX];
 #pragma unroll
         for (int e = 0; e < NMAX; ++e) {
-            acc[e] = warp_sum(acc[e]);
+            acc[e] = warp_sum(da[e].value(BF16));
             if (bias != nullptr && e < N)
                 acc[e] += static_cast<double>(bias[e]);
         }
@@ -141,53 +177,44 @@ __global__ void __launch_bounds__(kThreads)
                 val[j] = bv;
             }
         }
-        // full softmax over N (aux statistic p, and mode F gates)
+        // full softmax over N, one expert per lane (aux statistic p, mode F gates)
         const double mx = val[0];
-        double Z = 0.0;
-        double pe[NMAX];
-#pragma unroll
-        for (int e = 0; e < NMAX; ++e) {
-            pe[e] = (e < N) ? exp(acc[e] - mx) : 0.0;
-            Z += pe[e];
-        }
-#pragma unroll
-        for (int e = 0; e < NMAX; ++e) {
-            pe[e] /= Z;
-            psum[e] += pe[e];
-        }
-        double g[kMaxK];
-        double gs = 0.0;
-#pragma unroll
-        for (int j = 0; j < kMaxK; ++j) {
-            g[j] = 0.0;
-            if (j < k) {
-                if (gate_mode == MOE_GATE_TOPK_THEN_SOFTMAX) {
-                    g[j] = exp(val[j] - mx);
-                } else {
-                    double pj = 0.0;
-#pragma unroll
-                    for (int e = 0; e < NMAX; ++e)
-                        if (e == sel[j])
-                            pj = pe[e];
-                    g[j] = pj;
-                }
-                gs += g[j];
-            }
-        }
-        const bool norm = (gate_mode == MOE_GATE_TOPK_THEN_SOFTMAX) || renorm;
-#pragma unroll
-        for (int j = 0; j < kMaxK; ++j) {
-            if (j < k && lane == j) {
-                topk_idx[t * k + j] = sel[j];
-                topk_w[t * k + j] = static_cast<float>(norm ? g[j] / gs : g[j]);
-            }
-        }
-    }
-    if (lane == 0) {
+        double my_l = 0.0;
 #pragma unroll
         for (int e = 0; e < NMAX; ++e)
-            s_p[warp][e] = psum[e];
+            if (e == lane)
+                my_l = acc[e];
+        const double my_ev = (lane < N) ? exp(my_l - mx) : 0.0;
+        const double Z = warp_sum(my_ev);
+        const double my_p = my_ev / Z;
+        if (lane < NMAX)
+            my_psum += my_p;
+        // gates: lane j < k computes slot j
+        double gj = 0.0;
+        int sj = 0;
+#pragma unroll
+        for (int j = 0; j < kMaxK; ++j)
+            if (j == lane) {
+                sj = sel[j];
+                gj = val[j];
+            }
+        if (lane < k) {
+            if (gate_mode == MOE_GATE_TOPK_THEN_SOFTMAX)
+                gj = exp(gj - mx);
+            else
+                gj = exp(gj - mx) / Z;
+        } else {
+            gj = 0.0;
+        }
+        const double gs = warp_sum(gj);
+        const bool norm = (gate_mode == MOE_GATE_TOPK_THEN_SOFTMAX) || renorm;
+        if (lane < k) {
+            topk_idx[t * k + lane] = sj;
+            topk_w[t * k + lane] = static_cast<float>(norm ? gj / gs : gj);
+        }
     }
+    if (lane < NMAX)
+        s_p[warp][lane] = my_psum;
     __syncthreads();
     for (int e = threadIdx.x; e < N; e += kThreads) {
         double s = 0.0;
@@ -280,27 +307,27 @@ __global__ void __launch_bounds__(kThreads)
                     taken |= 1u << (be >> 5);
             }
         }
-        // fp64 recomputation of the candidates
-        double acc[kMaxCand];
-#pragma unroll
-        for (int c = 0; c < kMaxCand; ++c)
-            acc[c] = 0.0;
+        // recomputation of the candidates (compensated, see DotAcc)
+        DotAcc da[kMaxCand];
         const uint4 *xr = reinterpret_cast<const uint4 *>(x + t * static_cast<int64_t>(d) * esz);
+#pragma unroll 2
         for (int ch = lane; ch < chunks; ch += 32) {
-            const uint4 xa = __ldg(xr + ch);
+            float xf[8];
+            unpack_chunk<BF16>(__ldg(xr + ch), xf);
 #pragma unroll
             for (int c = 0; c < kMaxCand; ++c) {
                 if (c < KC) {
                     const uint4 wa = __ldg(reinterpret_cast<const uint4 *>(
                                                w + static_cast<int64_t>(cand[c]) * d * esz) +
                                            ch);
-                    acc[c] = chunk_dot<BF16>(xa, wa, acc[c]);
+                    chunk_dot<BF16>(xf, wa, da[c]);
                 }
             }
         }
+        double acc[kMaxCand];
 #pragma unroll
         for (int c = 0; c < kMaxCand; ++c) {
-            acc[c] = warp_sum(acc[c]);
+            acc[c] = warp_sum(da[c].value(BF16));
             if (bias != nullptr && c < KC)
                 acc[c] += static_cast<double>(bias[cand[c]]);
         }
@@ -380,15 +407,26 @@ __global__ void __launch_bounds__(kThreads)
     }
 }
 
-__global__ void p_finalize_kernel(const double *__restrict__ p_part, int nblk, int N, int64_t T,
-                                  float *__restrict__ p_mean)
+// p_mean[e] = (sum over router blocks b of p_part[b][e]) / T; one block per
+// expert, fixed-order tree so the result is the same on every run.
+__global__ void __launch_bounds__(256)
+    p_finalize_kernel(const double *__restrict__ p_part, int nblk, int N, int64_t T,
+                      float *__restrict__ p_mean)
 {
-    for (int e = blockIdx.x * blockDim.x + threadIdx.x; e < N; e += gridDim.x * blockDim.x) {
-        double s = 0.0;
-        for (int b = 0; b < nblk; ++b)
-            s += p_part[static_cast<int64_t>(b) * N + e];
-        p_mean[e] = T > 0 ? static_cast<float>(s / static_cast<double>(T)) : 0.0f;
+    __shared__ double s[256];
+    const int e = blockIdx.x;
+    double acc = 0.0;
+    for (int b = threadIdx.x; b < nblk; b += 256)
+        acc += p_part[static_cast<int64_t>(b) * N + e];
+    s[threadIdx.x] = acc;
+    __syncthreads();
+    for (int w = 128; w > 0; w >>= 1) {
+        if (threadIdx.x < w)
+            s[threadIdx.x] += s[threadIdx.x + w];
+        __syncthreads();
     }
+    if (threadIdx.x == 0)
+        p_mean[e] = T > 0 ? static_cast<float>(s[0] / static_cast<double>(T)) : 0.0f;
 }
 
 int router_grid(int64_t T)
@@ -455,7 +493,7 @@ cudaError_t launch_router_select(RouterLaunch &L, cudaStream_t stream)
 cudaError_t launch_p_finalize(const double *p_part, int32_t p_blocks, int32_t N, int64_t T,
                               float *p_mean, cudaStream_t stream)
 {
-    p_finalize_kernel<<<1, 256, 0, stream>>>(p_part, p_blocks, N, T, p_mean);
+    p_finalize_kernel<<<N, 256, 0, stream>>>(p_part, p_blocks, N, T, p_mean);
     count_launches(1);
     return cudaGetLastError();
 }
