@@ -146,6 +146,33 @@ moe_status moe_dispatch(const moe_config *cfg, const void *x, const int32_t *top
                         const float *p_mean, float *f, float *aux_loss,
                         void *workspace, size_t workspace_bytes, void *stream);
 
+/* Dispatch without a workspace, for callers that cannot allocate device
+ * memory for one: a host framework that owns all device memory through its
+ * own pool, or a runtime with a fixed memory budget set up front, or a call
+ * path where cudaMalloc/cudaFree are not acceptable because they may
+ * synchronise the device.  (The pages have no counterpart to this entry
+ * point; it is a deployment variant of moe_dispatch.)
+ *
+ * Arguments and results are those of moe_dispatch without the workspace.
+ * The scratch the dispatch kernels keep between their launches (per-block
+ * expert counts and a status word) lives instead in an array of about
+ * 128 KiB compiled into this library, which every GPU that loads the library
+ * holds until the process exits.  Limits: T*k <= 262144 pairs and N <= 256
+ * experts; larger calls return MOE_ERR_WORKSPACE before anything is enqueued.
+ * The library allocates nothing: no cudaMalloc, cudaFree or allocating
+ * library routine.  The first call on each device looks up the device
+ * address of the array (cudaGetSymbolAddress, with that device current), so
+ * make that first call before any stream capture.  All calls on one device
+ * share the array: calls that may run at the same time on the GPU (unordered
+ * streams, several host threads) race and must be serialised by the caller.
+ * An out-of-range expert index is dropped as in moe_dispatch but is not
+ * reported, since there is no workspace status word to read. */
+moe_status moe_dispatch_noalloc(const moe_config *cfg, const void *x, const int32_t *topk_idx,
+                                int32_t *expert_counts, int32_t *expert_offsets, int32_t *perm,
+                                int32_t *inv_row, uint8_t *drop_mask, void *x_perm,
+                                float *x_scale, const float *p_mean, float *f, float *aux_loss,
+                                void *stream);
+
 /* Stage 3, expert FFNs as one grouped GEMM ("MoE: what it costs to train and
  * serve", Expert parallelism step 2).
  *   x_perm         [T*k, d] dispatch_dtype (rows >= offsets[N] are ignored)

@@ -1,0 +1,94 @@
+"""moe_dispatch_noalloc against moe_dispatch.
+
+moe_dispatch_noalloc is the dispatch entry point for callers that cannot give
+the library a workspace allocated with cudaMalloc: a host framework that owns
+all device memory through its own pool, a runtime whose memory budget is
+fixed up front, or a call path where cudaMalloc/cudaFree may not be used
+because they can synchronise the device.  It keeps its scratch in an array
+built into the library instead.  This file is collected last so that a run
+that stops at the first failure has run every other test before it.
+
+Each case calls the no-allocation entry point twice in a row (the second time
+on different routing, so leftovers in the shared array would show) and
+compares both results with moe_dispatch given a workspace, bit for bit as the
+other dispatch tests do.
+"""
+import ctypes
+
+import numpy as np
+import pytest
+import torch
+
+import synth
+import top_routing_expert_warp_b200 as moe
+from gpu_util import cfg_of, tdtype, upload_inputs
+
+pytestmark = pytest.mark.gpu
+
+CASES = {
+    "capacity-bf16": synth.SWITCH.with_(T=1000, d=128, H=256),
+    "fp8-k8": synth.DEEPSEEK.with_(T=200, d=256, H=128, H_shared=128),
+    "fp32": synth.TINY_F32,
+}
+
+
+def _buffers(wl):
+    rows = wl.T * wl.k
+    fp8 = wl.dispatch == "fp8"
+    return dict(
+        counts=torch.empty(wl.N, dtype=torch.int32, device="cuda"),
+        offs=torch.empty(wl.N + 1, dtype=torch.int32, device="cuda"),
+        perm=torch.full((rows,), -1, dtype=torch.int32, device="cuda"),
+        inv=torch.empty(rows, dtype=torch.int32, device="cuda"),
+        drop=torch.empty(rows, dtype=torch.uint8, device="cuda"),
+        xp=torch.zeros((rows, wl.d), dtype=torch.uint8 if fp8 else tdtype(wl), device="cuda"),
+        xs=torch.zeros(rows, dtype=torch.float32, device="cuda") if fp8 else None,
+        f=torch.empty(wl.N, dtype=torch.float32, device="cuda"),
+        aux=torch.empty(1, dtype=torch.float32, device="cuda"),
+    )
+
+
+def _same(a, b, R):
+    assert torch.equal(a["counts"], b["counts"])
+    assert torch.equal(a["offs"], b["offs"])
+    assert torch.equal(a["perm"][:R], b["perm"][:R])
+    assert torch.equal(a["inv"], b["inv"])
+    assert torch.equal(a["drop"], b["drop"])
+    assert torch.equal(a["xp"][:R].view(torch.uint8), b["xp"][:R].view(torch.uint8))
+    if a["xs"] is not None:
+        assert torch.equal(a["xs"][:R], b["xs"][:R])
+    assert torch.equal(a["f"], b["f"])
+    assert torch.equal(a["aux"], b["aux"])
+
+
+@pytest.mark.parametrize("name", list(CASES))
+def test_noalloc_dispatch_matches_workspace_dispatch(name):
+    wl = CASES[name]
+    cfg = cfg_of(wl)
+    dev, _ = upload_inputs(wl)
+    pm = torch.full((wl.N,), 1.0 / wl.N, dtype=torch.float32, device="cuda")
+    ws = moe.workspace(cfg)
+    for call, skew in enumerate((0.6, 0.1)):
+        idx = torch.from_numpy(synth.synthetic_topk(wl.seed + 90 + call, wl.T, wl.N, wl.k,
+                                                    skew=skew)).cuda()
+        ref, got = _buffers(wl), _buffers(wl)
+        moe.moe_dispatch(cfg, dev["x"], idx, ref["counts"], ref["offs"], ref["perm"], ref["inv"],
+                         ref["drop"], ref["xp"], ref["xs"], pm, ref["f"], ref["aux"], ws)
+        moe.moe_dispatch_noalloc(cfg, dev["x"], idx, got["counts"], got["offs"], got["perm"],
+                                 got["inv"], got["drop"], got["xp"], got["xs"], pm, got["f"],
+                                 got["aux"])
+        torch.cuda.synchronize()
+        assert moe.moe_check_status(ws)[0] == moe.MOE_OK
+        R = int(ref["offs"][-1].item())
+        _same(ref, got, R)
+
+
+def test_noalloc_rejects_batches_beyond_its_scratch():
+    # 262145 (token, slot) pairs: one more than the built-in array holds
+    cfg = moe.make_config(262145, 128, 8, 1, 128)
+    fake = ctypes.c_void_p(1 << 40)          # never dereferenced: rejected on the host
+    r = moe.lib().moe_dispatch_noalloc(ctypes.byref(cfg), fake, fake, fake, fake, fake, fake,
+                                       fake, fake, None, None, None, None, None)
+    assert r == moe.MOE_ERR_WORKSPACE
+    ok = moe.make_config(131072, 128, 8, 2, 128)   # exactly at the limit: accepted sizes
+    assert ok.T * ok.k == 262144

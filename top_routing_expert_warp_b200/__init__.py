@@ -26,7 +26,8 @@ MOE_ACT_RELU, MOE_ACT_SWIGLU = 0, 1
 
 EXPORTS = ("moe_workspace_bytes", "moe_router", "moe_dispatch", "moe_expert_ffn", "moe_combine",
            "moe_layer_forward", "moe_check_status", "moe_status_string", "moe_last_error_string",
-           "moe_version", "moe_launch_count", "moe_profile_begin", "moe_profile_end")
+           "moe_version", "moe_launch_count", "moe_profile_begin", "moe_profile_end",
+           "moe_dispatch_noalloc")
 PROFILE_STAGES = ("router", "dispatch", "expert_up", "expert_down", "shared_expert", "combine")
 
 
@@ -66,6 +67,8 @@ def lib():
         L.moe_workspace_bytes.restype = ctypes.c_size_t
         L.moe_router.argtypes = [cfgp, P, P, P, P, P, P, P, P, ctypes.c_size_t, P]
         L.moe_dispatch.argtypes = [cfgp, P, P, P, P, P, P, P, P, P, P, P, P, P, ctypes.c_size_t, P]
+        L.moe_dispatch_noalloc.argtypes = [cfgp, P, P, P, P, P, P, P, P, P, P, P, P, P]
+        L.moe_dispatch_noalloc.restype = ctypes.c_int
         L.moe_expert_ffn.argtypes = [cfgp, P, P, P, P, P, P, P, P, ctypes.c_size_t, P]
         L.moe_combine.argtypes = [cfgp, P, P, P, P, P, P, ctypes.c_size_t, P]
         L.moe_layer_forward.argtypes = [cfgp, P, P, P, P, P, P, P, P, P, P, P, P, P, P, P, P, P,
@@ -158,6 +161,18 @@ def moe_dispatch(cfg, x, topk_idx, expert_counts, expert_offsets, perm, inv_row,
                               _ptr(workspace), workspace.numel() * workspace.element_size(),
                               _stream(stream)),
            "moe_dispatch")
+
+
+def moe_dispatch_noalloc(cfg, x, topk_idx, expert_counts, expert_offsets, perm, inv_row,
+                         drop_mask, x_perm, x_scale, p_mean, f, aux_loss, stream=None):
+    """moe_dispatch for callers that cannot allocate a workspace: the library's
+    built-in scratch array is used instead (T*k <= 262144, N <= 256; calls on
+    one device must not overlap on the GPU)."""
+    _check(lib().moe_dispatch_noalloc(ctypes.byref(cfg), _ptr(x), _ptr(topk_idx),
+                                      _ptr(expert_counts), _ptr(expert_offsets), _ptr(perm),
+                                      _ptr(inv_row), _ptr(drop_mask), _ptr(x_perm), _ptr(x_scale),
+                                      _ptr(p_mean), _ptr(f), _ptr(aux_loss), _stream(stream)),
+           "moe_dispatch_noalloc")
 
 
 def moe_expert_ffn(cfg, x_perm, x_scale, expert_offsets, W1, W3, W2, y_perm, workspace,
