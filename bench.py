@@ -51,6 +51,21 @@ def env_rank():
             int(os.environ.get("WORLD_SIZE", "1")))
 
 
+def max_over_ranks(value: float, dist, device) -> float:
+    """Max of a per-rank time over all ranks (the job is as slow as its slowest rank)."""
+    if dist is None:
+        return float(value)
+    import torch
+    t = torch.tensor([float(value)], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def weak_value(tokens_per_rank: int, world: int, ms_per_step: float) -> float:
+    """Whole-job tokens/s: every rank processes its own batch in the step time."""
+    return world * tokens_per_rank / (ms_per_step * 1e-3)
+
+
 def mult(wl):
     return 3 if wl.act == "swiglu" else 2
 
@@ -200,28 +215,42 @@ def oracle_sample(wl, budget_s: float, max_tokens: int = 4096):
 
 
 def run_reference(args, wl):
+    """The reference arm: the CPU oracle, timed as it stands on this host's cores.
+
+    Each step is the oracle forward of n evenly spaced tokens of the workload,
+    n chosen so that the whole --warmup + --steps run stays within a few
+    minutes.  Under torchrun only rank 0 runs; the other ranks exit at once."""
     rank, _, world = env_rank()
     if rank != 0:
         return 0
     cores = len(os.sched_getaffinity(0))
-    # size each step so the whole run stays within a few minutes
-    per_step_budget = min(2.0, 150.0 / max(1, args.steps + args.warmup))
-    rate0, n0, s0, desc = oracle_sample(wl, per_step_budget, max_tokens=8)
+    per_step_budget = min(1.0, 150.0 / max(1, args.steps + args.warmup))
+    _oracle_tokens(wl, 1)                      # builds the host inputs once
+    n = 1
+    while n < 64:
+        t0 = time.perf_counter()
+        _oracle_tokens(wl, 2 * n)
+        if time.perf_counter() - t0 > per_step_budget:
+            break
+        n *= 2
+    for _ in range(args.warmup):
+        _oracle_tokens(wl, n)
     times = []
-    for i in range(args.warmup + args.steps):
-        rate, n, s, _ = oracle_sample(wl, per_step_budget, max_tokens=8) if i == 0 else (None, n0, None, None)
-        if i >= args.warmup:
-            t0 = time.perf_counter()
-            _oracle_tokens(wl, n0)
-            times.append(time.perf_counter() - t0)
-    ms = 1000.0 * statistics.mean(times) if times else float("nan")
-    value = n0 / (ms / 1000.0)
+    for _ in range(args.steps):
+        t0 = time.perf_counter()
+        _oracle_tokens(wl, n)
+        times.append(time.perf_counter() - t0)
+    ms = 1000.0 * statistics.mean(times)
+    value = n / (ms / 1000.0)
+    desc = (f"each step: {n} of {wl.T} tokens (router, top-k, dispatch, expert FFN and combine "
+            f"of their {n * wl.k} rows; capacity not applied to the sample), fp64, {cores} host "
+            f"threads (OpenMP)")
     line = {"impl": "reference", "metric": METRIC, "value": value, "unit": "tokens/s",
             "n_gpus": world, "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms,
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
             "data": "synthetic", "config": config_of(wl),
             "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": cores, "kind": "oracle",
-                             "sample": f"each step: {desc}"},
+                             "sample": desc},
             "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0,
                     "d2h_bytes_per_step": 0}}
     print(json.dumps(line), flush=True)
@@ -352,11 +381,7 @@ def run_ours(args, wl):
     stages, nrec = moe.moe_profile_end()
     launches = moe.moe_launch_count() - l0
     barrier()
-    ms_total = e0.elapsed_time(e1)
-    if dist is not None:
-        t = torch.tensor([ms_total], device="cuda")
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        ms_total = float(t.item())
+    ms_total = max_over_ranks(e0.elapsed_time(e1), dist, "cuda")
     ms = ms_total / args.steps
     st, word = moe.moe_check_status(ws)
     if st != moe.MOE_OK:
@@ -379,12 +404,7 @@ def run_ours(args, wl):
     a1.record(stream)
     torch.cuda.synchronize()
     barrier()
-    e2e_ms = a0.elapsed_time(a1)
-    if dist is not None:
-        t = torch.tensor([e2e_ms], device="cuda")
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        e2e_ms = float(t.item())
-    e2e_ms /= e_steps
+    e2e_ms = max_over_ranks(a0.elapsed_time(a1), dist, "cuda") / e_steps
 
     pk, pk_src = peaks()
     out = None
@@ -430,13 +450,13 @@ def run_ours(args, wl):
             cpu = {"value": rate, "unit": "tokens/s", "cores": len(os.sched_getaffinity(0)),
                    "kind": "oracle", "sample": desc, "seconds": secs}
         clocks = clk.summary()
-        out = {"metric": METRIC, "value": world * wl.T / (ms * 1e-3), "unit": "tokens/s",
+        out = {"metric": METRIC, "value": weak_value(wl.T, world, ms), "unit": "tokens/s",
                "n_gpus": world, "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms,
                "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": wl.dtype,
                "data": "synthetic (seeded SplitMix64 + Box-Muller normals; weights N(0, 1/fan_in))",
                "config": config_of(wl), "roofline": roof, "layer_roofline": layer,
                "cpu_baseline": cpu,
-               "e2e": {"value": world * wl.T / (e2e_ms * 1e-3), "unit": "tokens/s",
+               "e2e": {"value": weak_value(wl.T, world, e2e_ms), "unit": "tokens/s",
                        "ms_per_step": e2e_ms,
                        "h2d_bytes_per_step": int(xs[0].numel() * xs[0].element_size()),
                        "d2h_bytes_per_step": int(y.numel() * y.element_size())},

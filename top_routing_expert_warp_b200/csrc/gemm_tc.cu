@@ -53,6 +53,8 @@ struct GemmParams {
     const float *row_scale;  // multiply each accumulator row by row_scale[r], or null
     int64_t rows_cap;        // rows allocated in out (and row_scale); rows beyond are never written
     int32_t prefetch;        // 1: prefetch weight boxes into L2 ahead of their loads
+    int32_t ksplit;          // >1: split K; split s writes its partial sums at out + s*split_stride
+    int64_t split_stride;    // elements
     uint32_t *status;
 };
 
@@ -81,12 +83,15 @@ struct TileInfo {
     int32_t g, row0, rows_valid, n0;
     bool swap;
     int32_t ntok;   // swapped tiles: MMA N (rows_valid rounded up to 16)
+    int32_t ks, kb0, kb1;   // K split index and its k-block range
 };
 
-// Locate tile t: prefix[g] <= t < prefix[g+1].
+// Locate tile t: prefix[g] <= t < prefix[g+1].  Inside a group the order is
+// (K split, n tile, m tile) with m fastest, so CTAs running side by side share
+// the weight tile through L2.
 __device__ __forceinline__ TileInfo tile_info(int t, const int32_t *s_prefix,
                                               const int32_t *s_off, int G, int n_tiles,
-                                              int outn)
+                                              int outn, int ksplit, int KB)
 {
     int lo = 0, hi = G;  // find largest g with prefix[g] <= t
     while (hi - lo > 1) {
@@ -100,6 +105,9 @@ __device__ __forceinline__ TileInfo tile_info(int t, const int32_t *s_prefix,
     int rows_g = s_off[g + 1] - s_off[g];
     int mt_g = (rows_g + BM - 1) / BM;
     int local = t - s_prefix[g];
+    const int per_split = mt_g * n_tiles;
+    const int ks = local / per_split;
+    local -= ks * per_split;
     int n_tile = local / mt_g;
     int m_tile = local - n_tile * mt_g;
     TileInfo ti;
@@ -109,7 +117,9 @@ __device__ __forceinline__ TileInfo tile_info(int t, const int32_t *s_prefix,
     ti.n0 = n_tile * outn;
     ti.swap = ti.rows_valid <= kSwapMaxRows;
     ti.ntok = (ti.rows_valid + 15) & ~15;
-    (void)n_tiles;
+    ti.ks = ks;
+    ti.kb0 = static_cast<int>((static_cast<int64_t>(ks) * KB) / ksplit);
+    ti.kb1 = static_cast<int>((static_cast<int64_t>(ks + 1) * KB) / ksplit);
     return ti;
 }
 
@@ -231,7 +241,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             if (g < G) {
                 int rows = s_off[g + 1] - s_off[g];
                 rows = rows > 0 ? rows : 0;
-                sum += ((rows + BM - 1) / BM) * n_tiles;
+                sum += ((rows + BM - 1) / BM) * n_tiles * p.ksplit;
             }
         }
         int incl = sum;
@@ -248,7 +258,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                 if (g < G) {
                     int rows = s_off[g + 1] - s_off[g];
                     rows = rows > 0 ? rows : 0;
-                    run += ((rows + BM - 1) / BM) * n_tiles;
+                    run += ((rows + BM - 1) / BM) * n_tiles * p.ksplit;
                 }
             }
         }
@@ -269,10 +279,12 @@ __global__ void __launch_bounds__(kThreads, 1)
             bool ok = true;
             // L2 prefetch cursor: kPrefetchAhead k-blocks ahead of the loads in
             // this CTA's own (tile, k-block) sequence, weights only
-            int pf_t = blockIdx.x, pf_kb = 0, pf_brow = 0;
+            int pf_t = blockIdx.x, pf_kb = 0, pf_kb1 = 0, pf_brow = 0;
             if (pf_t < total_tiles) {
-                const TileInfo pi = tile_info(pf_t, s_prefix, s_off, G, n_tiles, OUTN);
+                const TileInfo pi = tile_info(pf_t, s_prefix, s_off, G, n_tiles, OUTN, p.ksplit, KB);
                 pf_brow = pi.g * p.n_out + pi.n0;
+                pf_kb = pi.kb0;
+                pf_kb1 = pi.kb1;
             }
             auto prefetch_next = [&]() {
                 if (!p.prefetch || pf_t >= total_tiles)
@@ -280,24 +292,25 @@ __global__ void __launch_bounds__(kThreads, 1)
                 tma_prefetch_l2_2d(&tmB, pf_kb * BK, pf_brow);
                 if (EPI == EPI_SWIGLU)
                     tma_prefetch_l2_2d(&tmB2, pf_kb * BK, pf_brow);
-                if (++pf_kb == KB) {
-                    pf_kb = 0;
+                if (++pf_kb >= pf_kb1) {
                     pf_t += gridDim.x;
                     if (pf_t < total_tiles) {
-                        const TileInfo pi = tile_info(pf_t, s_prefix, s_off, G, n_tiles, OUTN);
+                        const TileInfo pi = tile_info(pf_t, s_prefix, s_off, G, n_tiles, OUTN, p.ksplit, KB);
                         pf_brow = pi.g * p.n_out + pi.n0;
+                        pf_kb = pi.kb0;
+                        pf_kb1 = pi.kb1;
                     }
                 }
             };
             for (int i = 0; i < kPrefetchAhead; ++i)
                 prefetch_next();
             for (int t = blockIdx.x; t < total_tiles && ok; t += gridDim.x) {
-                const TileInfo ti = tile_info(t, s_prefix, s_off, G, n_tiles, OUTN);
+                const TileInfo ti = tile_info(t, s_prefix, s_off, G, n_tiles, OUTN, p.ksplit, KB);
                 const int brow = ti.g * p.n_out + ti.n0;
                 const int a_boxes = ti.ntok / 16;          // swapped tile: 16-row boxes
                 const uint32_t bytes = ti.swap ? (a_boxes * 16 * BK * 2 + Geo::B_STAGE_BYTES)
                                                : Geo::STAGE_BYTES;
-                for (int kb = 0; kb < KB; ++kb) {
+                for (int kb = ti.kb0; kb < ti.kb1; ++kb) {
                     if (!mbar_wait_bounded(&empty[s], ph ^ 1u, s_abort)) {
                         set_status(p.status, DEV_TIMEOUT_PRODUCER);
                         *s_abort = 1;
@@ -347,7 +360,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             int it = 0;
             bool ok = true;
             for (int t = blockIdx.x; t < total_tiles && ok; t += gridDim.x, ++it) {
-                const TileInfo ti = tile_info(t, s_prefix, s_off, G, n_tiles, OUTN);
+                const TileInfo ti = tile_info(t, s_prefix, s_off, G, n_tiles, OUTN, p.ksplit, KB);
                 const uint32_t idesc_s = idesc_bf16_f32(128, ti.ntok);
                 const int a = it & 1;
                 const uint32_t aph = (it >> 1) & 1;
@@ -358,7 +371,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                 }
                 tc_fence_after();
                 const uint32_t d_tmem = tmem_base + a * BN;
-                for (int kb = 0; kb < KB; ++kb) {
+                for (int kb = ti.kb0; kb < ti.kb1; ++kb) {
                     if (!mbar_wait_bounded(&full[s], ph, s_abort)) {
                         set_status(p.status, DEV_TIMEOUT_MMA);
                         *s_abort = 1;
@@ -373,7 +386,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                         for (int kk = 0; kk < BK / 16; ++kk)
                             tc_mma_bf16(d_tmem, sdesc_kmajor_sw128(sa + kk * 32),
                                         sdesc_kmajor_sw128(sb + kk * 32), idesc_n,
-                                        (kb > 0 || kk > 0) ? 1u : 0u);
+                                        (kb > ti.kb0 || kk > 0) ? 1u : 0u);
                     } else {
                         // D^T: weight rows are the MMA's M, the tile's tokens its N
 #pragma unroll
@@ -383,7 +396,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                                 tc_mma_bf16(d_tmem + h * 128,
                                             sdesc_kmajor_sw128(sb + h * 128 * BK * 2 + kk * 32),
                                             sdesc_kmajor_sw128(sa + kk * 32), idesc_s,
-                                            (kb > 0 || kk > 0) ? 1u : 0u);
+                                            (kb > ti.kb0 || kk > 0) ? 1u : 0u);
                     }
                     tc_commit(&empty[s]);
                     if (++s == STAGES) {
@@ -401,7 +414,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         const int r_in_tile = q * 32 + lane;
         int it = 0;
         for (int t = blockIdx.x; t < total_tiles; t += gridDim.x, ++it) {
-            const TileInfo ti = tile_info(t, s_prefix, s_off, G, n_tiles, OUTN);
+            const TileInfo ti = tile_info(t, s_prefix, s_off, G, n_tiles, OUTN, p.ksplit, KB);
             const int a = it & 1;
             const uint32_t aph = (it >> 1) & 1;
             const bool got = mbar_wait_bounded(&acc_full[a], aph, s_abort);
@@ -443,7 +456,8 @@ __global__ void __launch_bounds__(kThreads, 1)
                         }
                     }
                     if (row_ok)
-                        store_row32<OUT_F32>(p.out, row * p.ld_out, ti.n0 + c, p.n_out, o);
+                        store_row32<OUT_F32>(p.out, ti.ks * p.split_stride + row * p.ld_out,
+                                             ti.n0 + c, p.n_out, o);
                 }
             } else {
                 // swapped tile: lane = output feature, columns = tokens
@@ -468,7 +482,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                             const float o = silu_f(__uint_as_float(v[i]) * sc[i]) *
                                             (__uint_as_float(u[i]) * sc[i]);
                             if (c + i < ti.rows_valid && row < p.rows_cap && col < p.n_out)
-                                store_one<OUT_F32>(p.out, row * p.ld_out + col, o);
+                                store_one<OUT_F32>(p.out, ti.ks * p.split_stride + row * p.ld_out + col, o);
                         }
                     } else {
 #pragma unroll
@@ -484,7 +498,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                                 if (EPI == EPI_RELU)
                                     x = fmaxf(x, 0.0f);
                                 if (c + i < ti.rows_valid && row < p.rows_cap && col < p.n_out)
-                                    store_one<OUT_F32>(p.out, row * p.ld_out + col, x);
+                                    store_one<OUT_F32>(p.out, ti.ks * p.split_stride + row * p.ld_out + col, x);
                             }
                         }
                     }
@@ -603,11 +617,13 @@ cudaError_t launch_impl(const GemmLaunch &L, cudaStream_t stream)
     p.row_scale = L.row_scale;
     p.rows_cap = L.out_rows;
     p.prefetch = L.prefetch;
+    p.ksplit = L.ksplit > 1 ? L.ksplit : 1;
+    p.split_stride = L.split_stride;
     p.status = L.status;
     const int outn = Geo::OUTN;
     const int64_t n_tiles = (L.n_out + outn - 1) / outn;
     const int64_t m_tiles_max = (L.a_rows + BM - 1) / BM + (L.offsets ? L.G : 0);
-    int64_t tiles_max = n_tiles * m_tiles_max;
+    int64_t tiles_max = n_tiles * m_tiles_max * p.ksplit;
     int grid = static_cast<int>(tiles_max < sm_count() ? tiles_max : sm_count());
     if (grid <= 0)
         return cudaSuccess;
@@ -618,6 +634,19 @@ cudaError_t launch_impl(const GemmLaunch &L, cudaStream_t stream)
 }
 
 }  // namespace
+
+int router_ksplit(int64_t T, int32_t N, int32_t d)
+{
+    const int64_t m_tiles = (T + BM - 1) / BM;
+    const int64_t KB = (d + BK - 1) / BK;
+    (void)N;  // one n tile (N <= 256)
+    int64_t ks = (sm_count() + m_tiles - 1) / m_tiles;
+    if (ks > kRouterMaxSplit)
+        ks = kRouterMaxSplit;
+    if (ks > KB)
+        ks = KB;
+    return ks < 1 ? 1 : static_cast<int>(ks);
+}
 
 cudaError_t launch_grouped_gemm(const GemmLaunch &L, cudaStream_t stream)
 {

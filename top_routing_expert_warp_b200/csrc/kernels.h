@@ -31,8 +31,13 @@ struct GemmLaunch {
     int64_t ld_out;
     const float *row_scale;  // [a_rows] or null
     int32_t prefetch;        // prefetch weight boxes into L2 ahead of their loads
+    int32_t ksplit;          // >1: K split into ksplit slices (fp32 partial outputs)
+    int64_t split_stride;    // elements between the partial outputs of two slices
     uint32_t *status;
 };
+// K slices the router GEMM uses so that its tiles cover the SMs.
+int router_ksplit(int64_t T, int32_t N, int32_t d);
+constexpr int kRouterMaxSplit = 8;
 cudaError_t launch_grouped_gemm(const GemmLaunch &L, cudaStream_t stream);
 
 // fp32 CUDA-core grouped GEMM (fp32 layers): see ffn_simt.cu.
@@ -50,7 +55,8 @@ struct RouterLaunch {
     int64_t T;
     int32_t d, N, k;
     int32_t gate_mode, renormalize;
-    const float *logits_in;  // large-N path: fp32 logits from the tensor-core GEMM
+    const float *logits_in;  // large-N path: fp32 partial logits [ksplit][T][N] from the GEMM
+    int32_t ksplit;          // number of partial logit slices
     float *logits_out;       // optional fp32 logits (small-N path)
     int32_t *topk_idx;
     float *topk_w;

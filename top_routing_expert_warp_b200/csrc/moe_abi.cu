@@ -111,7 +111,8 @@ Layout layout_of(const moe_config &c)
     };
     L.status = take(256);
     L.p_part = take(static_cast<size_t>(moe::kRouterMaxBlocks) * N * sizeof(double));
-    L.logits = take(N > static_cast<size_t>(moe::kRouterSmallMaxN) ? T * N * 4 : 0);
+    L.logits = take(N > static_cast<size_t>(moe::kRouterSmallMaxN)
+                        ? static_cast<size_t>(moe::kRouterMaxSplit) * T * N * 4 : 0);
     L.topk_idx = take(rows * 4);
     L.topk_w = take(rows * 4);
     L.p_mean = take(N * 4);
@@ -186,7 +187,10 @@ moe_status run_router(const moe_config &c, const void *x, const void *Wg, const 
         R.logits_out = logits;
         MOE_CUDA(moe::launch_router_small(R, s));
     } else {
-        float *lg = logits ? logits : w.at<float>(w.L.logits);
+        // logits = sum of ksplit fp32 partial GEMMs over slices of d (so the
+        // tiles cover the SMs), summed in slice order by the selection kernel
+        float *part = w.at<float>(w.L.logits);
+        const int ks = moe::router_ksplit(c.T, c.N, c.d);
         moe::GemmLaunch G{};
         G.epi = moe::EPI_STORE;
         G.out_f32 = true;
@@ -200,13 +204,17 @@ moe_status run_router(const moe_config &c, const void *x, const void *Wg, const 
         G.rows_single = static_cast<int32_t>(c.T);
         G.G = 1;
         G.n_out = c.N;
-        G.out = lg;
+        G.out = part;
         G.out_rows = c.T;
         G.ld_out = c.N;
         G.row_scale = nullptr;
+        G.ksplit = ks;
+        G.split_stride = c.T * c.N;
         G.status = w.status();
         MOE_CUDA(moe::launch_grouped_gemm(G, s));
-        R.logits_in = lg;
+        R.logits_in = part;
+        R.ksplit = ks;
+        R.logits_out = logits;
         MOE_CUDA(moe::launch_router_select(R, s));
     }
     if (p_mean)

@@ -106,6 +106,76 @@ __device__ __forceinline__ void unpack_chunk(const uint4 a, float (&xf)[8])
     }
 }
 
+// Selection and gates of one token from its N logits (fp64, every lane holds
+// all of them).  Lane e accumulates the softmax probability of expert e into
+// *my_psum.
+template <int NMAX>
+__device__ __forceinline__ void small_select(const double (&acc)[NMAX], int64_t t, int N, int k,
+                                             int gate_mode, int renorm, int lane,
+                                             int32_t *__restrict__ topk_idx,
+                                             float *__restrict__ topk_w, double *my_psum)
+{
+    // top-k: strict comparison in ascending expert order -> lowest index wins
+    uint32_t taken = 0;
+    int sel[kMaxK];
+    double val[kMaxK];
+#pragma unroll
+    for (int j = 0; j < kMaxK; ++j) {
+        sel[j] = 0;
+        val[j] = 0.0;
+        if (j < k) {
+            int bi = -1;
+            double bv = 0.0;
+#pragma unroll
+            for (int e = 0; e < NMAX; ++e) {
+                if (e < N && !((taken >> e) & 1u) && (bi < 0 || acc[e] > bv)) {
+                    bi = e;
+                    bv = acc[e];
+                }
+            }
+            taken |= 1u << bi;
+            sel[j] = bi;
+            val[j] = bv;
+        }
+    }
+    // full softmax over N, one expert per lane (aux statistic p, mode F gates)
+    const double mx = val[0];
+    double my_l = 0.0;
+#pragma unroll
+    for (int e = 0; e < NMAX; ++e)
+        if (e == lane)
+            my_l = acc[e];
+    const double my_ev = (lane < N) ? exp(my_l - mx) : 0.0;
+    const double Z = warp_sum(my_ev);
+    *my_psum += my_ev / Z;
+    // gates: lane j < k computes slot j
+    double gj = 0.0;
+    int sj = 0;
+#pragma unroll
+    for (int j = 0; j < kMaxK; ++j)
+        if (j == lane) {
+            sj = sel[j];
+            gj = val[j];
+        }
+    if (lane < k)
+        gj = (gate_mode == MOE_GATE_TOPK_THEN_SOFTMAX) ? exp(gj - mx) : exp(gj - mx) / Z;
+    else
+        gj = 0.0;
+    const double gs = warp_sum(gj);
+    const bool norm = (gate_mode == MOE_GATE_TOPK_THEN_SOFTMAX) || renorm;
+    if (lane < k) {
+        topk_idx[t * k + lane] = sj;
+        topk_w[t * k + lane] = static_cast<float>(norm ? gj / gs : gj);
+    }
+}
+
+// Small-N router: a warp takes kTokPerWarp tokens at a time and kUnroll
+// 16-byte chunks per lane per pass, so several loads of x (from HBM) and of
+// W_g (L1-resident) are in flight per lane and each W_g chunk serves every
+// token of the warp.
+constexpr int kTokPerWarp = 2;
+constexpr int kUnroll = 4;
+
 template <bool BF16, int NMAX>
 __global__ void __launch_bounds__(kThreads)
     router_small_kernel(const void *__restrict__ xv, const void *__restrict__ wv,
@@ -120,97 +190,68 @@ __global__ void __launch_bounds__(kThreads)
     const int chunks = d * esz / 16;
     const uint8_t *x = static_cast<const uint8_t *>(xv);
     const uint8_t *w = static_cast<const uint8_t *>(wv);
-
     double my_psum = 0.0;  // lane e: this warp's sum of p_e over its tokens
 
-    for (int64_t t = static_cast<int64_t>(blockIdx.x) * kWarps + warp; t < T;
-         t += static_cast<int64_t>(gridDim.x) * kWarps) {
-        DotAcc da[NMAX];
-        const uint4 *xr = reinterpret_cast<const uint4 *>(x + t * static_cast<int64_t>(d) * esz);
-#pragma unroll 2
-        for (int c = lane; c < chunks; c += 32) {
-            float xf[8];
-            unpack_chunk<BF16>(__ldg(xr + c), xf);
+    const int64_t step = static_cast<int64_t>(gridDim.x) * kWarps * kTokPerWarp;
+    for (int64_t t0 = (static_cast<int64_t>(blockIdx.x) * kWarps + warp) * kTokPerWarp; t0 < T;
+         t0 += step) {
+        DotAcc da[kTokPerWarp][NMAX];
+        const uint4 *xr[kTokPerWarp];
+#pragma unroll
+        for (int q = 0; q < kTokPerWarp; ++q) {
+            const int64_t tq = (t0 + q < T) ? t0 + q : t0;   // a missing token re-reads t0
+            xr[q] = reinterpret_cast<const uint4 *>(x + tq * static_cast<int64_t>(d) * esz);
+        }
+        for (int c0 = lane; c0 < chunks; c0 += 32 * kUnroll) {
+            float xf[kTokPerWarp][kUnroll][8];
+#pragma unroll
+            for (int u = 0; u < kUnroll; ++u) {
+                const int c = c0 + 32 * u;
+#pragma unroll
+                for (int q = 0; q < kTokPerWarp; ++q) {
+                    uint4 v = make_uint4(0, 0, 0, 0);
+                    if (c < chunks)
+                        v = __ldg(xr[q] + c);
+                    unpack_chunk<BF16>(v, xf[q][u]);
+                }
+            }
 #pragma unroll
             for (int e = 0; e < NMAX; ++e) {
                 if (e < N) {
-                    const uint4 wa = __ldg(reinterpret_cast<const uint4 *>(
-                                               w + static_cast<int64_t>(e) * d * esz) +
-                                           c);
-                    chunk_dot<BF16>(xf, wa, da[e]);
-                }
-            }
-        }
-        double acc[NMAX];
+                    const uint4 *wr = reinterpret_cast<const uint4 *>(
+                        w + static_cast<int64_t>(e) * d * esz);
 #pragma unroll
-        for (int e = 0; e < NMAX; ++e) {
-            acc[e] = warp_sum(da[e].value(BF16));
-            if (bias != nullptr && e < N)
-                acc[e] += static_cast<double>(bias[e]);
-        }
-        if (logits_out != nullptr) {
+                    for (int u = 0; u < kUnroll; ++u) {
+                        const int c = c0 + 32 * u;
+                        if (c < chunks) {
+                            const uint4 wa = __ldg(wr + c);
 #pragma unroll
-            for (int e = 0; e < NMAX; ++e)
-                if (e < N && lane == e)
-                    logits_out[t * N + e] = static_cast<float>(acc[e]);
-        }
-        // top-k: strict comparison in ascending expert order -> lowest index wins
-        uint32_t taken = 0;
-        int sel[kMaxK];
-        double val[kMaxK];
-#pragma unroll
-        for (int j = 0; j < kMaxK; ++j) {
-            sel[j] = 0;
-            val[j] = 0.0;
-            if (j < k) {
-                int bi = -1;
-                double bv = 0.0;
-#pragma unroll
-                for (int e = 0; e < NMAX; ++e) {
-                    if (e < N && !((taken >> e) & 1u) && (bi < 0 || acc[e] > bv)) {
-                        bi = e;
-                        bv = acc[e];
+                            for (int q = 0; q < kTokPerWarp; ++q)
+                                chunk_dot<BF16>(xf[q][u], wa, da[q][e]);
+                        }
                     }
                 }
-                taken |= 1u << bi;
-                sel[j] = bi;
-                val[j] = bv;
             }
         }
-        // full softmax over N, one expert per lane (aux statistic p, mode F gates)
-        const double mx = val[0];
-        double my_l = 0.0;
 #pragma unroll
-        for (int e = 0; e < NMAX; ++e)
-            if (e == lane)
-                my_l = acc[e];
-        const double my_ev = (lane < N) ? exp(my_l - mx) : 0.0;
-        const double Z = warp_sum(my_ev);
-        const double my_p = my_ev / Z;
-        if (lane < NMAX)
-            my_psum += my_p;
-        // gates: lane j < k computes slot j
-        double gj = 0.0;
-        int sj = 0;
+        for (int q = 0; q < kTokPerWarp; ++q) {
+            const int64_t t = t0 + q;
+            double acc[NMAX];
 #pragma unroll
-        for (int j = 0; j < kMaxK; ++j)
-            if (j == lane) {
-                sj = sel[j];
-                gj = val[j];
+            for (int e = 0; e < NMAX; ++e) {
+                acc[e] = warp_sum(da[q][e].value(BF16));
+                if (bias != nullptr && e < N)
+                    acc[e] += static_cast<double>(bias[e]);
             }
-        if (lane < k) {
-            if (gate_mode == MOE_GATE_TOPK_THEN_SOFTMAX)
-                gj = exp(gj - mx);
-            else
-                gj = exp(gj - mx) / Z;
-        } else {
-            gj = 0.0;
-        }
-        const double gs = warp_sum(gj);
-        const bool norm = (gate_mode == MOE_GATE_TOPK_THEN_SOFTMAX) || renorm;
-        if (lane < k) {
-            topk_idx[t * k + lane] = sj;
-            topk_w[t * k + lane] = static_cast<float>(norm ? gj / gs : gj);
+            if (t >= T)
+                continue;
+            if (logits_out != nullptr) {
+#pragma unroll
+                for (int e = 0; e < NMAX; ++e)
+                    if (e < N && lane == e)
+                        logits_out[t * N + e] = static_cast<float>(acc[e]);
+            }
+            small_select<NMAX>(acc, t, N, k, gate_mode, renorm, lane, topk_idx, topk_w, &my_psum);
         }
     }
     if (lane < NMAX)
@@ -232,7 +273,8 @@ __device__ __forceinline__ bool better(float v1, int e1, float v2, int e2)
 
 template <bool BF16>
 __global__ void __launch_bounds__(kThreads)
-    router_select_kernel(float *__restrict__ logits, const void *__restrict__ xv,
+    router_select_kernel(const float *__restrict__ part, int ksplit,
+                         float *__restrict__ logits_out, const void *__restrict__ xv,
                          const void *__restrict__ wv, const float *__restrict__ bias, int64_t T,
                          int d, int N, int k, int gate_mode, int renorm,
                          int32_t *__restrict__ topk_idx, float *__restrict__ topk_w,
@@ -267,11 +309,14 @@ __global__ void __launch_bounds__(kThreads)
             const int e = lane + 32 * i;
             lv[i] = -INFINITY;
             if (i < npl && e < N) {
-                float v = logits[t * N + e];
-                if (bias != nullptr) {
+                // partial logits of the K slices, summed in slice order
+                float v = 0.0f;
+                for (int sl = 0; sl < ksplit; ++sl)
+                    v += part[static_cast<int64_t>(sl) * T * N + t * N + e];
+                if (bias != nullptr)
                     v += bias[e];
-                    logits[t * N + e] = v;
-                }
+                if (logits_out != nullptr)
+                    logits_out[t * N + e] = v;
                 lv[i] = v;
             }
         }
@@ -307,20 +352,28 @@ __global__ void __launch_bounds__(kThreads)
                     taken |= 1u << (be >> 5);
             }
         }
-        // recomputation of the candidates (compensated, see DotAcc)
+        // recomputation of the candidates (compensated, see DotAcc), kUnroll
+        // chunks of x in flight per lane
         DotAcc da[kMaxCand];
         const uint4 *xr = reinterpret_cast<const uint4 *>(x + t * static_cast<int64_t>(d) * esz);
-#pragma unroll 2
-        for (int ch = lane; ch < chunks; ch += 32) {
-            float xf[8];
-            unpack_chunk<BF16>(__ldg(xr + ch), xf);
+        for (int c0 = lane; c0 < chunks; c0 += 32 * kUnroll) {
+            float xf[kUnroll][8];
+#pragma unroll
+            for (int u = 0; u < kUnroll; ++u) {
+                const int ch = c0 + 32 * u;
+                unpack_chunk<BF16>(ch < chunks ? __ldg(xr + ch) : make_uint4(0, 0, 0, 0), xf[u]);
+            }
 #pragma unroll
             for (int c = 0; c < kMaxCand; ++c) {
                 if (c < KC) {
-                    const uint4 wa = __ldg(reinterpret_cast<const uint4 *>(
-                                               w + static_cast<int64_t>(cand[c]) * d * esz) +
-                                           ch);
-                    chunk_dot<BF16>(xf, wa, da[c]);
+                    const uint4 *wr = reinterpret_cast<const uint4 *>(
+                        w + static_cast<int64_t>(cand[c]) * d * esz);
+#pragma unroll
+                    for (int u = 0; u < kUnroll; ++u) {
+                        const int ch = c0 + 32 * u;
+                        if (ch < chunks)
+                            chunk_dot<BF16>(xf[u], __ldg(wr + ch), da[c]);
+                    }
                 }
             }
         }
@@ -429,9 +482,9 @@ __global__ void __launch_bounds__(256)
         p_mean[e] = T > 0 ? static_cast<float>(s[0] / static_cast<double>(T)) : 0.0f;
 }
 
-int router_grid(int64_t T)
+int router_grid(int64_t T, int tok_per_warp)
 {
-    int64_t want = (T + kWarps - 1) / kWarps;
+    int64_t want = (T + kWarps * tok_per_warp - 1) / (kWarps * tok_per_warp);
     int sms = 148;
     int dev = 0;
     if (cudaGetDevice(&dev) == cudaSuccess)
@@ -448,7 +501,7 @@ int router_grid(int64_t T)
 
 cudaError_t launch_router_small(RouterLaunch &L, cudaStream_t stream)
 {
-    const int grid = router_grid(L.T);
+    const int grid = router_grid(L.T, kTokPerWarp);
     *L.p_blocks = grid;
     if (L.dtype == MOE_BF16) {
         if (L.N <= 8)
@@ -475,16 +528,16 @@ cudaError_t launch_router_small(RouterLaunch &L, cudaStream_t stream)
 
 cudaError_t launch_router_select(RouterLaunch &L, cudaStream_t stream)
 {
-    const int grid = router_grid(L.T);
+    const int grid = router_grid(L.T, 1);
     *L.p_blocks = grid;
     const size_t smem = static_cast<size_t>(kWarps) * L.N * sizeof(double);
     if (L.dtype == MOE_BF16)
         router_select_kernel<true><<<grid, kThreads, smem, stream>>>(
-            const_cast<float *>(L.logits_in), L.x, L.Wg, L.bias, L.T, L.d, L.N, L.k,
+            L.logits_in, L.ksplit, L.logits_out, L.x, L.Wg, L.bias, L.T, L.d, L.N, L.k,
             L.gate_mode, L.renormalize, L.topk_idx, L.topk_w, L.p_part);
     else
         router_select_kernel<false><<<grid, kThreads, smem, stream>>>(
-            const_cast<float *>(L.logits_in), L.x, L.Wg, L.bias, L.T, L.d, L.N, L.k,
+            L.logits_in, L.ksplit, L.logits_out, L.x, L.Wg, L.bias, L.T, L.d, L.N, L.k,
             L.gate_mode, L.renormalize, L.topk_idx, L.topk_w, L.p_part);
     count_launches(1);
     return cudaGetLastError();
