@@ -121,3 +121,20 @@ def test_ragged_rows_many_tiles():
     wl = synth.Workload("ragged", T=300, d=192, N=1, k=1, H=256, act="swiglu", dtype="bf16",
                         gate_mode="R", seed=25)
     _layer_vs_oracle(wl)
+
+
+@pytest.mark.parametrize("act", ["swiglu", "relu"])
+def test_pair_tiles_ragged(act):
+    # >= 512 rows per expert selects the CTA-pair GEMM (256-row tiles); segments
+    # of ~550 rows end in partial pair tiles and H = 384 masks output columns
+    wl = synth.Workload("pair", T=1100, d=256, N=2, k=1, H=384, act=act, dtype="bf16",
+                        gate_mode="R", seed=26)
+    run, ref = _layer_vs_oracle(wl)
+    assert ref["R"] >= 512 * wl.N // 2 and np.all(ref["kept"] > 256)
+
+
+def test_pair_tiles_shared_expert():
+    # the shared expert runs every token (1100 rows, one group) on CTA pairs
+    wl = synth.Workload("pair-shared", T=1100, d=256, N=4, k=1, H=128, act="swiglu",
+                        dtype="bf16", gate_mode="F", renormalize=True, H_shared=256, seed=27)
+    _layer_vs_oracle(wl)

@@ -39,6 +39,11 @@ struct GemmLaunch {
 int router_ksplit(int64_t T, int32_t N, int32_t d);
 constexpr int kRouterMaxSplit = 8;
 cudaError_t launch_grouped_gemm(const GemmLaunch &L, cudaStream_t stream);
+// Same contract on CTA pairs (256-row tiles, tcgen05 cta_group::2), bf16 output,
+// no K split: see gemm_tc2.cu.  For compute-bound shapes (many rows per group).
+cudaError_t launch_grouped_gemm_pair(const GemmLaunch &L, cudaStream_t stream);
+// Rows per group from which the pair kernel is used.
+constexpr int64_t kPairMinRowsPerGroup = 512;
 
 // fp32 CUDA-core grouped GEMM (fp32 layers): see ffn_simt.cu.
 cudaError_t launch_simt_gemm_f32(int epi, const float *A, int64_t rows_cap, int32_t K,

@@ -307,7 +307,9 @@ moe_status run_ffn(const moe_config &c, const void *A, const float *row_scale, i
     U.ld_out = H;
     U.row_scale = row_scale;
     U.status = status;
-    MOE_CUDA(moe::launch_grouped_gemm(U, s));
+    // compute-bound expert projections (many rows per expert) run on CTA pairs
+    const bool pair = rows_cap >= moe::kPairMinRowsPerGroup * G;
+    MOE_CUDA(pair ? moe::launch_grouped_gemm_pair(U, s) : moe::launch_grouped_gemm(U, s));
     if (mark_between >= 0)
         prof_mark(mark_between, s);
     moe::GemmLaunch Dn{};
@@ -328,7 +330,7 @@ moe_status run_ffn(const moe_config &c, const void *A, const float *row_scale, i
     Dn.ld_out = c.d;
     Dn.row_scale = nullptr;
     Dn.status = status;
-    MOE_CUDA(moe::launch_grouped_gemm(Dn, s));
+    MOE_CUDA(pair ? moe::launch_grouped_gemm_pair(Dn, s) : moe::launch_grouped_gemm(Dn, s));
     return MOE_OK;
 }
 
