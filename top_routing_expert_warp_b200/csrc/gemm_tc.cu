@@ -641,8 +641,9 @@ int router_ksplit(int64_t T, int32_t N, int32_t d)
     const int64_t KB = (d + BK - 1) / BK;
     (void)N;  // one n tile (N <= 256)
     int64_t ks = (sm_count() + m_tiles - 1) / m_tiles;
-    if (ks > kRouterMaxSplit)
-        ks = kRouterMaxSplit;
+    const int64_t cap = router_ksplit_cap(T, N);
+    if (ks > cap)
+        ks = cap;
     if (ks > KB)
         ks = KB;
     return ks < 1 ? 1 : static_cast<int>(ks);

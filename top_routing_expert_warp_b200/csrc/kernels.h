@@ -35,9 +35,21 @@ struct GemmLaunch {
     int64_t split_stride;    // elements between the partial outputs of two slices
     uint32_t *status;
 };
-// K slices the router GEMM uses so that its tiles cover the SMs.
+// K slices the router GEMM uses so that its tiles cover the SMs, at most
+// router_ksplit_cap(T, N) (which sizes the workspace's partial-logit buffer).
 int router_ksplit(int64_t T, int32_t N, int32_t d);
-constexpr int kRouterMaxSplit = 8;
+constexpr int kRouterMaxSplit = 32;
+constexpr int64_t kRouterPartialBudget = int64_t(1) << 24;   // fp32 partial logits
+inline int router_ksplit_cap(int64_t T, int32_t N)
+{
+    const int64_t tn = T * N;
+    if (tn <= 0)
+        return 1;
+    int64_t c = kRouterPartialBudget / tn;
+    if (c > kRouterMaxSplit)
+        c = kRouterMaxSplit;
+    return c < 1 ? 1 : static_cast<int>(c);
+}
 cudaError_t launch_grouped_gemm(const GemmLaunch &L, cudaStream_t stream);
 // Same contract on CTA pairs (256-row tiles, tcgen05 cta_group::2), bf16 output,
 // no K split: see gemm_tc2.cu.  For compute-bound shapes (many rows per group).

@@ -111,8 +111,8 @@ Layout layout_of(const moe_config &c)
     };
     L.status = take(256);
     L.p_part = take(static_cast<size_t>(moe::kRouterMaxBlocks) * N * sizeof(double));
-    L.logits = take(N > static_cast<size_t>(moe::kRouterSmallMaxN)
-                        ? static_cast<size_t>(moe::kRouterMaxSplit) * T * N * 4 : 0);
+    L.logits = take(c.dtype == MOE_BF16
+                        ? static_cast<size_t>(moe::router_ksplit_cap(c.T, c.N)) * T * N * 4 : 0);
     L.topk_idx = take(rows * 4);
     L.topk_w = take(rows * 4);
     L.p_mean = take(N * 4);
@@ -183,7 +183,8 @@ moe_status run_router(const moe_config &c, const void *x, const void *Wg, const 
     R.p_part = w.at<double>(w.L.p_part);
     R.p_blocks = &blocks;
     R.status = w.status();
-    if (c.N <= moe::kRouterSmallMaxN) {
+    if (c.dtype == MOE_F32) {
+        // fp32 layers (small N): CUDA cores, exact fp64 products
         R.logits_out = logits;
         MOE_CUDA(moe::launch_router_small(R, s));
     } else {

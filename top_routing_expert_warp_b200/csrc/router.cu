@@ -271,35 +271,66 @@ __device__ __forceinline__ bool better(float v1, int e1, float v2, int e2)
     return (v1 > v2) || (v1 == v2 && e1 < e2 && e1 >= 0) || (e2 < 0 && e1 >= 0);
 }
 
-template <bool BF16>
-__global__ void __launch_bounds__(kThreads)
+// Compensated fp32 accumulator (hi + lo) of bf16 dot products; see DotAcc.
+struct Comp {
+    float hi = 0.0f, lo = 0.0f;
+    __device__ __forceinline__ void add(float s)
+    {
+        const float t = hi + s;
+        const float bp = t - hi;
+        lo += (hi - (t - bp)) + (s - bp);
+        hi = t;
+    }
+};
+
+__device__ __forceinline__ float chunk_dot8(const float (&xf)[8], const uint4 b)
+{
+    const uint32_t bv[4] = {b.x, b.y, b.z, b.w};
+    float s = xf[0] * __uint_as_float(bv[0] << 16);
+    s = fmaf(xf[1], __uint_as_float(bv[0] & 0xFFFF0000u), s);
+#pragma unroll
+    for (int i = 1; i < 4; ++i) {
+        s = fmaf(xf[2 * i], __uint_as_float(bv[i] << 16), s);
+        s = fmaf(xf[2 * i + 1], __uint_as_float(bv[i] & 0xFFFF0000u), s);
+    }
+    return s;
+}
+
+// Selection from the tensor-core logits (bf16 layers, any N <= 256): one warp
+// per token.  The logits are the K-slice partial sums of the router GEMM,
+// added in slice order.  The KC best become candidates; their logits are
+// recomputed from x and W_g with exact products and compensated sums, the
+// candidates are re-ranked on those values (descending, lower index first)
+// and the gates are taken from them.  The full softmax for p (aux loss) uses
+// the recomputed candidates and fp32 exponentials of the other logits.
+constexpr int kSelUnroll = 2;
+
+__global__ void __launch_bounds__(kThreads, 2)
     router_select_kernel(const float *__restrict__ part, int ksplit,
-                         float *__restrict__ logits_out, const void *__restrict__ xv,
-                         const void *__restrict__ wv, const float *__restrict__ bias, int64_t T,
+                         float *__restrict__ logits_out, const uint16_t *__restrict__ x,
+                         const uint16_t *__restrict__ w, const float *__restrict__ bias, int64_t T,
                          int d, int N, int k, int gate_mode, int renorm,
                          int32_t *__restrict__ topk_idx, float *__restrict__ topk_w,
                          double *__restrict__ p_part)
 {
     extern __shared__ double s_pdyn[];  // [kWarps][N]
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    const int esz = BF16 ? 2 : 4;
-    const int chunks = d * esz / 16;
-    const uint8_t *x = static_cast<const uint8_t *>(xv);
-    const uint8_t *w = static_cast<const uint8_t *>(wv);
+    const int chunks = d / 8;
     const int npl = (N + 31) / 32;
+    // candidates recomputed at fp64-level accuracy: the k selected experts,
+    // whose logits alone set the gates in modes R and renormalised F; two more
+    // in plain mode F, whose softmax denominator also weighs the runners-up
     const bool mode_f_raw = (gate_mode == MOE_GATE_SOFTMAX_THEN_TOPK) && !renorm;
-    int KC = k + 2;
-    if (mode_f_raw && KC < 8)
-        KC = 8;
+    int KC = mode_f_raw ? k + 2 : k;
     if (KC > N)
         KC = N;
     if (KC > kMaxCand)
         KC = kMaxCand;
 
-    double psum[kMaxPerLane];
+    float psum[kMaxPerLane];
 #pragma unroll
     for (int i = 0; i < kMaxPerLane; ++i)
-        psum[i] = 0.0;
+        psum[i] = 0.0f;
 
     for (int64_t t = static_cast<int64_t>(blockIdx.x) * kWarps + warp; t < T;
          t += static_cast<int64_t>(gridDim.x) * kWarps) {
@@ -309,8 +340,7 @@ __global__ void __launch_bounds__(kThreads)
             const int e = lane + 32 * i;
             lv[i] = -INFINITY;
             if (i < npl && e < N) {
-                // partial logits of the K slices, summed in slice order
-                float v = 0.0f;
+                float v = 0.0f;  // K-slice partial logits, summed in slice order
                 for (int sl = 0; sl < ksplit; ++sl)
                     v += part[static_cast<int64_t>(sl) * T * N + t * N + e];
                 if (bias != nullptr)
@@ -320,7 +350,7 @@ __global__ void __launch_bounds__(kThreads)
                 lv[i] = v;
             }
         }
-        // candidates: the KC best fp32 logits, best first
+        // candidates: the KC best logits, best first
         int cand[kMaxCand];
         uint32_t taken = 0;
 #pragma unroll
@@ -332,8 +362,7 @@ __global__ void __launch_bounds__(kThreads)
 #pragma unroll
                 for (int i = 0; i < kMaxPerLane; ++i) {
                     const int e = lane + 32 * i;
-                    if (i < npl && e < N && !((taken >> i) & 1u) &&
-                        (be < 0 || lv[i] > bv)) {
+                    if (i < npl && e < N && !((taken >> i) & 1u) && (be < 0 || lv[i] > bv)) {
                         bv = lv[i];
                         be = e;
                     }
@@ -352,27 +381,26 @@ __global__ void __launch_bounds__(kThreads)
                     taken |= 1u << (be >> 5);
             }
         }
-        // recomputation of the candidates (compensated, see DotAcc), kUnroll
-        // chunks of x in flight per lane
-        DotAcc da[kMaxCand];
-        const uint4 *xr = reinterpret_cast<const uint4 *>(x + t * static_cast<int64_t>(d) * esz);
-        for (int c0 = lane; c0 < chunks; c0 += 32 * kUnroll) {
-            float xf[kUnroll][8];
+        // recomputation of the candidates
+        Comp da[kMaxCand];
+        const uint4 *xr = reinterpret_cast<const uint4 *>(x + t * static_cast<int64_t>(d));
+        for (int c0 = lane; c0 < chunks; c0 += 32 * kSelUnroll) {
+            float xf[kSelUnroll][8];
 #pragma unroll
-            for (int u = 0; u < kUnroll; ++u) {
+            for (int u = 0; u < kSelUnroll; ++u) {
                 const int ch = c0 + 32 * u;
-                unpack_chunk<BF16>(ch < chunks ? __ldg(xr + ch) : make_uint4(0, 0, 0, 0), xf[u]);
+                unpack_chunk<true>(ch < chunks ? __ldg(xr + ch) : make_uint4(0, 0, 0, 0), xf[u]);
             }
 #pragma unroll
             for (int c = 0; c < kMaxCand; ++c) {
                 if (c < KC) {
-                    const uint4 *wr = reinterpret_cast<const uint4 *>(
-                        w + static_cast<int64_t>(cand[c]) * d * esz);
+                    const uint4 *wr =
+                        reinterpret_cast<const uint4 *>(w + static_cast<int64_t>(cand[c]) * d);
 #pragma unroll
-                    for (int u = 0; u < kUnroll; ++u) {
+                    for (int u = 0; u < kSelUnroll; ++u) {
                         const int ch = c0 + 32 * u;
                         if (ch < chunks)
-                            chunk_dot<BF16>(xf[u], __ldg(wr + ch), da[c]);
+                            da[c].add(chunk_dot8(xf[u], __ldg(wr + ch)));
                     }
                 }
             }
@@ -380,11 +408,11 @@ __global__ void __launch_bounds__(kThreads)
         double acc[kMaxCand];
 #pragma unroll
         for (int c = 0; c < kMaxCand; ++c) {
-            acc[c] = warp_sum(da[c].value(BF16));
+            acc[c] = warp_sum(static_cast<double>(da[c].hi) + static_cast<double>(da[c].lo));
             if (bias != nullptr && c < KC)
                 acc[c] += static_cast<double>(bias[cand[c]]);
         }
-        // order candidates by (fp64 value desc, index asc); fixed-shape
+        // order candidates by (recomputed value desc, index asc); fixed-shape
         // exchange sort so that every index is a compile-time constant
 #pragma unroll
         for (int pass = 0; pass < kMaxCand - 1; ++pass) {
@@ -405,51 +433,56 @@ __global__ void __launch_bounds__(kThreads)
             }
         }
         const double mx = acc[0];
-        // full softmax over N: candidates use fp64 logits, the rest fp32 ones
-        double Z = 0.0;
-        double ev[kMaxPerLane];
+        const float mxf = static_cast<float>(mx);
+        // softmax denominator: candidates in fp64, the others in fp32
+        float ev[kMaxPerLane];
+        double zl = 0.0;
 #pragma unroll
         for (int i = 0; i < kMaxPerLane; ++i) {
             const int e = lane + 32 * i;
-            ev[i] = 0.0;
+            ev[i] = 0.0f;
             if (i < npl && e < N) {
-                double l = static_cast<double>(lv[i]);
+                double ce = -1.0;
 #pragma unroll
                 for (int c = 0; c < kMaxCand; ++c)
                     if (c < KC && cand[c] == e)
-                        l = acc[c];
-                ev[i] = exp(l - mx);
-                Z += ev[i];
+                        ce = exp(acc[c] - mx);
+                if (ce >= 0.0) {
+                    zl += ce;
+                    ev[i] = static_cast<float>(ce);
+                } else {
+                    ev[i] = expf(lv[i] - mxf);
+                    zl += static_cast<double>(ev[i]);
+                }
             }
         }
-        Z = warp_sum(Z);
+        const double Z = warp_sum(zl);
+        const float zinv = static_cast<float>(1.0 / Z);
 #pragma unroll
         for (int i = 0; i < kMaxPerLane; ++i)
-            psum[i] += ev[i] / Z;
-        double g[kMaxK];
-        double gs = 0.0;
+            psum[i] += ev[i] * zinv;
+        // gates: lane j < k computes slot j from the recomputed logits
+        double aj = 0.0;
+        int ej = 0;
 #pragma unroll
-        for (int j = 0; j < kMaxK; ++j) {
-            g[j] = 0.0;
-            if (j < k) {
-                g[j] = exp(acc[j] - mx);
-                gs += g[j];
+        for (int c = 0; c < kMaxCand; ++c)
+            if (c == lane) {
+                aj = acc[c];
+                ej = cand[c];
             }
-        }
+        double gj = (lane < k) ? exp(aj - mx) : 0.0;
+        const double gs = warp_sum(gj);
         const bool norm = (gate_mode == MOE_GATE_TOPK_THEN_SOFTMAX) || renorm;
-#pragma unroll
-        for (int j = 0; j < kMaxK; ++j) {
-            if (j < k && lane == j) {
-                topk_idx[t * k + j] = cand[j];
-                topk_w[t * k + j] = static_cast<float>(norm ? g[j] / gs : g[j] / Z);
-            }
+        if (lane < k) {
+            topk_idx[t * k + lane] = ej;
+            topk_w[t * k + lane] = static_cast<float>(norm ? gj / gs : gj / Z);
         }
     }
 #pragma unroll
     for (int i = 0; i < kMaxPerLane; ++i) {
         const int e = lane + 32 * i;
         if (i < npl && e < N)
-            s_pdyn[warp * N + e] = psum[i];
+            s_pdyn[warp * N + e] = static_cast<double>(psum[i]);
     }
     __syncthreads();
     for (int e = threadIdx.x; e < N; e += kThreads) {
@@ -489,7 +522,7 @@ int router_grid(int64_t T, int tok_per_warp)
     int dev = 0;
     if (cudaGetDevice(&dev) == cudaSuccess)
         cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
-    int64_t cap = static_cast<int64_t>(sms) * 4;
+    int64_t cap = static_cast<int64_t>(sms) * 8;
     if (cap > kRouterMaxBlocks)
         cap = kRouterMaxBlocks;
     if (want > cap)
@@ -528,17 +561,15 @@ cudaError_t launch_router_small(RouterLaunch &L, cudaStream_t stream)
 
 cudaError_t launch_router_select(RouterLaunch &L, cudaStream_t stream)
 {
+    if (L.dtype != MOE_BF16 || L.N > 32 * kMaxPerLane || L.k > kMaxCand)
+        return cudaErrorInvalidValue;
     const int grid = router_grid(L.T, 1);
     *L.p_blocks = grid;
     const size_t smem = static_cast<size_t>(kWarps) * L.N * sizeof(double);
-    if (L.dtype == MOE_BF16)
-        router_select_kernel<true><<<grid, kThreads, smem, stream>>>(
-            L.logits_in, L.ksplit, L.logits_out, L.x, L.Wg, L.bias, L.T, L.d, L.N, L.k,
-            L.gate_mode, L.renormalize, L.topk_idx, L.topk_w, L.p_part);
-    else
-        router_select_kernel<false><<<grid, kThreads, smem, stream>>>(
-            L.logits_in, L.ksplit, L.logits_out, L.x, L.Wg, L.bias, L.T, L.d, L.N, L.k,
-            L.gate_mode, L.renormalize, L.topk_idx, L.topk_w, L.p_part);
+    router_select_kernel<<<grid, kThreads, smem, stream>>>(
+        L.logits_in, L.ksplit, L.logits_out, static_cast<const uint16_t *>(L.x),
+        static_cast<const uint16_t *>(L.Wg), L.bias, L.T, L.d, L.N, L.k, L.gate_mode,
+        L.renormalize, L.topk_idx, L.topk_w, L.p_part);
     count_launches(1);
     return cudaGetLastError();
 }
