@@ -305,6 +305,10 @@ __device__ __forceinline__ float chunk_dot8(const float (&xf)[8], const uint4 b)
 // the recomputed candidates and fp32 exponentials of the other logits.
 constexpr int kSelUnroll = 2;
 
+// NPL: logits per lane (N <= 32 NPL); KCM: bound on the candidate count.
+// Both are compile-time so that every loop below has a fixed trip count and
+// the instantiation used by a layer stays small.
+template <int NPL, int KCM>
 __global__ void __launch_bounds__(kThreads, 2)
     router_select_kernel(const float *__restrict__ part, int ksplit,
                          float *__restrict__ logits_out, const uint16_t *__restrict__ x,
@@ -316,7 +320,6 @@ __global__ void __launch_bounds__(kThreads, 2)
     extern __shared__ double s_pdyn[];  // [kWarps][N]
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int chunks = d / 8;
-    const int npl = (N + 31) / 32;
     // candidates recomputed at fp64-level accuracy: the k selected experts,
     // whose logits alone set the gates in modes R and renormalised F; two more
     // in plain mode F, whose softmax denominator also weighs the runners-up
@@ -324,22 +327,22 @@ __global__ void __launch_bounds__(kThreads, 2)
     int KC = mode_f_raw ? k + 2 : k;
     if (KC > N)
         KC = N;
-    if (KC > kMaxCand)
-        KC = kMaxCand;
+    if (KC > KCM)
+        KC = KCM;
 
-    float psum[kMaxPerLane];
+    float psum[NPL];
 #pragma unroll
-    for (int i = 0; i < kMaxPerLane; ++i)
+    for (int i = 0; i < NPL; ++i)
         psum[i] = 0.0f;
 
     for (int64_t t = static_cast<int64_t>(blockIdx.x) * kWarps + warp; t < T;
          t += static_cast<int64_t>(gridDim.x) * kWarps) {
-        float lv[kMaxPerLane];
+        float lv[NPL];
 #pragma unroll
-        for (int i = 0; i < kMaxPerLane; ++i) {
+        for (int i = 0; i < NPL; ++i) {
             const int e = lane + 32 * i;
             lv[i] = -INFINITY;
-            if (i < npl && e < N) {
+            if (e < N) {
                 float v = 0.0f;  // K-slice partial logits, summed in slice order
                 for (int sl = 0; sl < ksplit; ++sl)
                     v += part[static_cast<int64_t>(sl) * T * N + t * N + e];
@@ -351,18 +354,18 @@ __global__ void __launch_bounds__(kThreads, 2)
             }
         }
         // candidates: the KC best logits, best first
-        int cand[kMaxCand];
+        int cand[KCM];
         uint32_t taken = 0;
 #pragma unroll
-        for (int c = 0; c < kMaxCand; ++c) {
+        for (int c = 0; c < KCM; ++c) {
             cand[c] = 0;
             if (c < KC) {
                 float bv = -INFINITY;
                 int be = -1;
 #pragma unroll
-                for (int i = 0; i < kMaxPerLane; ++i) {
+                for (int i = 0; i < NPL; ++i) {
                     const int e = lane + 32 * i;
-                    if (i < npl && e < N && !((taken >> i) & 1u) && (be < 0 || lv[i] > bv)) {
+                    if (e < N && !((taken >> i) & 1u) && (be < 0 || lv[i] > bv)) {
                         bv = lv[i];
                         be = e;
                     }
@@ -382,7 +385,7 @@ __global__ void __launch_bounds__(kThreads, 2)
             }
         }
         // recomputation of the candidates
-        Comp da[kMaxCand];
+        Comp da[KCM];
         const uint4 *xr = reinterpret_cast<const uint4 *>(x + t * static_cast<int64_t>(d));
         for (int c0 = lane; c0 < chunks; c0 += 32 * kSelUnroll) {
             float xf[kSelUnroll][8];
@@ -392,7 +395,7 @@ __global__ void __launch_bounds__(kThreads, 2)
                 unpack_chunk<true>(ch < chunks ? __ldg(xr + ch) : make_uint4(0, 0, 0, 0), xf[u]);
             }
 #pragma unroll
-            for (int c = 0; c < kMaxCand; ++c) {
+            for (int c = 0; c < KCM; ++c) {
                 if (c < KC) {
                     const uint4 *wr =
                         reinterpret_cast<const uint4 *>(w + static_cast<int64_t>(cand[c]) * d);
@@ -405,9 +408,9 @@ __global__ void __launch_bounds__(kThreads, 2)
                 }
             }
         }
-        double acc[kMaxCand];
+        double acc[KCM];
 #pragma unroll
-        for (int c = 0; c < kMaxCand; ++c) {
+        for (int c = 0; c < KCM; ++c) {
             acc[c] = warp_sum(static_cast<double>(da[c].hi) + static_cast<double>(da[c].lo));
             if (bias != nullptr && c < KC)
                 acc[c] += static_cast<double>(bias[cand[c]]);
@@ -415,10 +418,12 @@ __global__ void __launch_bounds__(kThreads, 2)
         // order candidates by (recomputed value desc, index asc); fixed-shape
         // exchange sort so that every index is a compile-time constant
 #pragma unroll
-        for (int pass = 0; pass < kMaxCand - 1; ++pass) {
+        for (int pass = 0; pass < KCM - 1; ++pass) {
+            if (pass + 1 >= KC)
+                break;
 #pragma unroll
-            for (int c = 0; c + 1 < kMaxCand; ++c) {
-                if (c + 1 < KC) {
+            for (int c = 0; c + 1 < KCM - pass; ++c) {
+                if (c + 1 < KC - pass) {
                     const bool sw = (acc[c] < acc[c + 1]) ||
                                     (acc[c] == acc[c + 1] && cand[c] > cand[c + 1]);
                     if (sw) {
@@ -435,16 +440,16 @@ __global__ void __launch_bounds__(kThreads, 2)
         const double mx = acc[0];
         const float mxf = static_cast<float>(mx);
         // softmax denominator: candidates in fp64, the others in fp32
-        float ev[kMaxPerLane];
+        float ev[NPL];
         double zl = 0.0;
 #pragma unroll
-        for (int i = 0; i < kMaxPerLane; ++i) {
+        for (int i = 0; i < NPL; ++i) {
             const int e = lane + 32 * i;
             ev[i] = 0.0f;
-            if (i < npl && e < N) {
+            if (e < N) {
                 double ce = -1.0;
 #pragma unroll
-                for (int c = 0; c < kMaxCand; ++c)
+                for (int c = 0; c < KCM; ++c)
                     if (c < KC && cand[c] == e)
                         ce = exp(acc[c] - mx);
                 if (ce >= 0.0) {
@@ -459,13 +464,13 @@ __global__ void __launch_bounds__(kThreads, 2)
         const double Z = warp_sum(zl);
         const float zinv = static_cast<float>(1.0 / Z);
 #pragma unroll
-        for (int i = 0; i < kMaxPerLane; ++i)
+        for (int i = 0; i < NPL; ++i)
             psum[i] += ev[i] * zinv;
         // gates: lane j < k computes slot j from the recomputed logits
         double aj = 0.0;
         int ej = 0;
 #pragma unroll
-        for (int c = 0; c < kMaxCand; ++c)
+        for (int c = 0; c < KCM; ++c)
             if (c == lane) {
                 aj = acc[c];
                 ej = cand[c];
@@ -479,9 +484,9 @@ __global__ void __launch_bounds__(kThreads, 2)
         }
     }
 #pragma unroll
-    for (int i = 0; i < kMaxPerLane; ++i) {
+    for (int i = 0; i < NPL; ++i) {
         const int e = lane + 32 * i;
-        if (i < npl && e < N)
+        if (e < N)
             s_pdyn[warp * N + e] = static_cast<double>(psum[i]);
     }
     __syncthreads();
@@ -559,6 +564,26 @@ cudaError_t launch_router_small(RouterLaunch &L, cudaStream_t stream)
     return cudaGetLastError();
 }
 
+template <int NPL, int KCM>
+void select_launch(RouterLaunch &L, int grid, size_t smem, cudaStream_t stream)
+{
+    router_select_kernel<NPL, KCM><<<grid, kThreads, smem, stream>>>(
+        L.logits_in, L.ksplit, L.logits_out, static_cast<const uint16_t *>(L.x),
+        static_cast<const uint16_t *>(L.Wg), L.bias, L.T, L.d, L.N, L.k, L.gate_mode,
+        L.renormalize, L.topk_idx, L.topk_w, L.p_part);
+}
+
+template <int NPL>
+void select_launch_kc(RouterLaunch &L, int kc, int grid, size_t smem, cudaStream_t stream)
+{
+    if (kc <= 2)
+        select_launch<NPL, 2>(L, grid, smem, stream);
+    else if (kc <= 4)
+        select_launch<NPL, 4>(L, grid, smem, stream);
+    else
+        select_launch<NPL, kMaxCand>(L, grid, smem, stream);
+}
+
 cudaError_t launch_router_select(RouterLaunch &L, cudaStream_t stream)
 {
     if (L.dtype != MOE_BF16 || L.N > 32 * kMaxPerLane || L.k > kMaxCand)
@@ -566,10 +591,18 @@ cudaError_t launch_router_select(RouterLaunch &L, cudaStream_t stream)
     const int grid = router_grid(L.T, 1);
     *L.p_blocks = grid;
     const size_t smem = static_cast<size_t>(kWarps) * L.N * sizeof(double);
-    router_select_kernel<<<grid, kThreads, smem, stream>>>(
-        L.logits_in, L.ksplit, L.logits_out, static_cast<const uint16_t *>(L.x),
-        static_cast<const uint16_t *>(L.Wg), L.bias, L.T, L.d, L.N, L.k, L.gate_mode,
-        L.renormalize, L.topk_idx, L.topk_w, L.p_part);
+    const bool mode_f_raw = (L.gate_mode == MOE_GATE_SOFTMAX_THEN_TOPK) && !L.renormalize;
+    int kc = mode_f_raw ? L.k + 2 : L.k;
+    if (kc > L.N)
+        kc = L.N;
+    if (L.N <= 32)
+        select_launch_kc<1>(L, kc, grid, smem, stream);
+    else if (L.N <= 64)
+        select_launch_kc<2>(L, kc, grid, smem, stream);
+    else if (L.N <= 128)
+        select_launch_kc<4>(L, kc, grid, smem, stream);
+    else
+        select_launch_kc<kMaxPerLane>(L, kc, grid, smem, stream);
     count_launches(1);
     return cudaGetLastError();
 }
