@@ -52,10 +52,24 @@ __global__ void __launch_bounds__(kThreads)
             row[j] = __shfl_sync(0xffffffffu, my_row, j);
             g[j] = __shfl_sync(0xffffffffu, my_g, j);
         }
-        // U chunks per lane per pass, so U loads per row are in flight at once
-        constexpr int U = 4;
+        // U chunks per lane per pass; the loads of every slot are issued
+        // before any is used (predicated, no branches), so k * U loads per
+        // lane are in flight at once
+        constexpr int U = 2;
         constexpr int V = BF16 ? 8 : 4;
         for (int c0 = lane; c0 < chunks; c0 += 32 * U) {
+            uint4 v[kMaxK][U];
+#pragma unroll
+            for (int j = 0; j < kMaxK; ++j) {
+                const uint4 *src = reinterpret_cast<const uint4 *>(
+                    y_perm + static_cast<int64_t>(row[j] > 0 ? row[j] : 0) * d * esz);
+#pragma unroll
+                for (int u = 0; u < U; ++u) {
+                    const int c = c0 + 32 * u;
+                    v[j][u] = (j < k && row[j] >= 0 && c < chunks) ? __ldg(src + c)
+                                                                   : make_uint4(0, 0, 0, 0);
+                }
+            }
             float acc[U][V];
 #pragma unroll
             for (int u = 0; u < U; ++u)
@@ -65,17 +79,9 @@ __global__ void __launch_bounds__(kThreads)
 #pragma unroll
             for (int j = 0; j < kMaxK; ++j) {
                 if (j < k && row[j] >= 0) {
-                    const uint4 *src = reinterpret_cast<const uint4 *>(
-                        y_perm + static_cast<int64_t>(row[j]) * d * esz);
-                    uint4 v[U];
 #pragma unroll
                     for (int u = 0; u < U; ++u) {
-                        const int c = c0 + 32 * u;
-                        v[u] = c < chunks ? __ldg(src + c) : make_uint4(0, 0, 0, 0);
-                    }
-#pragma unroll
-                    for (int u = 0; u < U; ++u) {
-                        const uint32_t w[4] = {v[u].x, v[u].y, v[u].z, v[u].w};
+                        const uint32_t w[4] = {v[j][u].x, v[j][u].y, v[j][u].z, v[j][u].w};
                         if (BF16) {
 #pragma unroll
                             for (int i = 0; i < 4; ++i) {

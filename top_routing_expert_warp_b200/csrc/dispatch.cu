@@ -313,6 +313,88 @@ __global__ void __launch_bounds__(kThreads)
     }
 }
 
+// Per-token FP8 payload for the fused layer path: scale = amax / 448 (1 for
+// an all-zero row) and code = E4M3(x / scale) as in the gather kernel above;
+// writes the codes' values as bf16 (exact) for the expert GEMM, which gathers
+// token rows directly, and the per-token scale for its epilogue.
+__global__ void __launch_bounds__(kThreads)
+    quantize_tokens_kernel(const uint8_t *__restrict__ x, int64_t T, int d,
+                           __nv_bfloat16 *__restrict__ xq, float *__restrict__ scale_out)
+{
+    const int lane = threadIdx.x & 31;
+    const int64_t nwarps = static_cast<int64_t>(gridDim.x) * kWarps;
+    const int chunks = d / 8;
+    for (int64_t t = static_cast<int64_t>(blockIdx.x) * kWarps + (threadIdx.x >> 5); t < T;
+         t += nwarps) {
+        const uint4 *src = reinterpret_cast<const uint4 *>(x + t * static_cast<int64_t>(d) * 2);
+        float amax = 0.0f;
+        for (int c = lane; c < chunks; c += 32) {
+            const uint4 v = __ldg(src + c);
+            const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+            for (int i = 0; i < 4; ++i) {
+                amax = fmaxf(amax, fabsf(__uint_as_float(w[i] << 16)));
+                amax = fmaxf(amax, fabsf(__uint_as_float(w[i] & 0xFFFF0000u)));
+            }
+        }
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1)
+            amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, o));
+        const float scale = amax > 0.0f ? __fdiv_rn(amax, 448.0f) : 1.0f;
+        if (lane == 0)
+            scale_out[t] = scale;
+        uint4 *dst = reinterpret_cast<uint4 *>(xq + t * static_cast<int64_t>(d));
+        for (int c = lane; c < chunks; c += 32) {
+            const uint4 v = __ldg(src + c);
+            const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+            uint32_t b[4];
+#pragma unroll
+            for (int i = 0; i < 4; ++i) {
+                __nv_fp8_e4m3 lo, hi;
+                lo.__x = __nv_cvt_float_to_fp8(__fdiv_rn(__uint_as_float(w[i] << 16), scale),
+                                               __NV_SATFINITE, __NV_E4M3);
+                hi.__x = __nv_cvt_float_to_fp8(__fdiv_rn(__uint_as_float(w[i] & 0xFFFF0000u), scale),
+                                               __NV_SATFINITE, __NV_E4M3);
+                b[i] = pack_bf16x2(static_cast<float>(lo), static_cast<float>(hi));
+            }
+            dst[c] = make_uint4(b[0], b[1], b[2], b[3]);
+        }
+    }
+}
+
+// Expert-ordered bf16 rows and row scales from the per-token FP8 payload.
+__global__ void __launch_bounds__(kThreads)
+    gather_quantized_kernel(const uint8_t *__restrict__ xq, const float *__restrict__ scale,
+                            int d, int k, const int32_t *__restrict__ perm,
+                            const int32_t *__restrict__ R_ptr, uint8_t *__restrict__ out,
+                            float *__restrict__ out_scale)
+{
+    const int lane = threadIdx.x & 31;
+    const int64_t R = *R_ptr;
+    const int64_t nwarps = static_cast<int64_t>(gridDim.x) * kWarps;
+    const int chunks = d / 8;
+    for (int64_t r = static_cast<int64_t>(blockIdx.x) * kWarps + (threadIdx.x >> 5); r < R;
+         r += nwarps) {
+        const int64_t t = perm[r] / k;
+        if (lane == 0)
+            out_scale[r] = scale[t];
+        const uint4 *src = reinterpret_cast<const uint4 *>(xq + t * static_cast<int64_t>(d) * 2);
+        uint4 *dst = reinterpret_cast<uint4 *>(out + r * static_cast<int64_t>(d) * 2);
+        constexpr int U = 4;
+        for (int c0 = lane; c0 < chunks; c0 += 32 * U) {
+            uint4 v[U];
+#pragma unroll
+            for (int u = 0; u < U; ++u)
+                if (c0 + 32 * u < chunks)
+                    v[u] = __ldg(src + c0 + 32 * u);
+#pragma unroll
+            for (int u = 0; u < U; ++u)
+                if (c0 + 32 * u < chunks)
+                    dst[c0 + 32 * u] = v[u];
+        }
+    }
+}
+
 int gather_grid(int64_t rows)
 {
     int sms = 148, dev = 0;
@@ -340,6 +422,10 @@ cudaError_t launch_dispatch(const DispatchLaunch &L, cudaStream_t stream)
                                                  L.aux_alpha);
     dispatch_rank_kernel<<<nblk, kThreads, kWarps * L.N * sizeof(int32_t), stream>>>(
         L.topk_idx, n_pairs, L.N, L.capacity, L.block_base, L.offsets, L.perm, L.inv_row, L.drop);
+    if (L.x_perm == nullptr) {      // the caller builds the expert-ordered rows itself
+        count_launches(3);
+        return cudaGetLastError();
+    }
     const int grid = gather_grid(n_pairs);
     const uint8_t *x = static_cast<const uint8_t *>(L.x);
     uint8_t *xp = static_cast<uint8_t *>(L.x_perm);
@@ -354,6 +440,30 @@ cudaError_t launch_dispatch(const DispatchLaunch &L, cudaStream_t stream)
             x, L.d, L.k, L.perm, L.offsets + L.N, xp, L.x_scale,
             static_cast<__nv_bfloat16 *>(L.x_bf16_copy));
     count_launches(4);
+    return cudaGetLastError();
+}
+
+cudaError_t launch_quantize_tokens(const void *x, int64_t T, int32_t d, void *xq, float *scale,
+                                   cudaStream_t stream)
+{
+    if (T == 0)
+        return cudaSuccess;
+    quantize_tokens_kernel<<<gather_grid(T), kThreads, 0, stream>>>(
+        static_cast<const uint8_t *>(x), T, d, static_cast<__nv_bfloat16 *>(xq), scale);
+    count_launches(1);
+    return cudaGetLastError();
+}
+
+cudaError_t launch_gather_quantized(const void *xq, const float *scale, int64_t T, int32_t d,
+                                    int32_t k, const int32_t *perm, const int32_t *offsets,
+                                    int32_t N, void *out, float *out_scale, cudaStream_t stream)
+{
+    if (T == 0)
+        return cudaSuccess;
+    gather_quantized_kernel<<<gather_grid(T * k), kThreads, 0, stream>>>(
+        static_cast<const uint8_t *>(xq), scale, d, k, perm, offsets + N,
+        static_cast<uint8_t *>(out), out_scale);
+    count_launches(1);
     return cudaGetLastError();
 }
 
