@@ -29,6 +29,7 @@ __global__ void __launch_bounds__(kThreads)
                    uint8_t *__restrict__ y, int64_t T, int d, int k, int64_t rows_cap,
                    uint32_t *status)
 {
+    grid_dep_wait();
     const int lane = threadIdx.x & 31;
     const int esz = BF16 ? 2 : 4;
     const int chunks = d * esz / 16;
@@ -152,12 +153,12 @@ cudaError_t launch_combine(int dtype, const void *y_perm, const int32_t *inv_row
         grid = static_cast<int64_t>(sms) * 8;
     const int64_t rows_cap = T * k;
     if (dtype == MOE_BF16)
-        combine_kernel<true><<<static_cast<int>(grid), kThreads, 0, stream>>>(
+        launch_k(combine_kernel<true>, static_cast<int>(grid), kThreads, 0, stream, 
             static_cast<const uint8_t *>(y_perm), inv_row, topk_w,
             static_cast<const uint8_t *>(y_shared), static_cast<uint8_t *>(y), T, d, k, rows_cap,
             status);
     else
-        combine_kernel<false><<<static_cast<int>(grid), kThreads, 0, stream>>>(
+        launch_k(combine_kernel<false>, static_cast<int>(grid), kThreads, 0, stream, 
             static_cast<const uint8_t *>(y_perm), inv_row, topk_w,
             static_cast<const uint8_t *>(y_shared), static_cast<uint8_t *>(y), T, d, k, rows_cap,
             status);

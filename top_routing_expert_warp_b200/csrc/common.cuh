@@ -40,6 +40,14 @@ __device__ __forceinline__ void set_status(uint32_t *status, uint32_t bits)
         atomicOr(status, bits);
 }
 
+// Programmatic dependent launch: wait until the previous kernel on the stream
+// has completed and its memory operations are visible (no-op when the kernel
+// was launched without the attribute).
+__device__ __forceinline__ void grid_dep_wait()
+{
+    asm volatile("griddepcontrol.wait;" ::: "memory");
+}
+
 // ------------------------------------------------------------------ smem
 __device__ __forceinline__ uint32_t smem_u32(const void *p)
 {

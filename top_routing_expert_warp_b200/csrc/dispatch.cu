@@ -41,6 +41,7 @@ __global__ void __launch_bounds__(kThreads)
     dispatch_count_kernel(const int32_t *__restrict__ idx, int64_t n_pairs, int N,
                           int32_t *__restrict__ block_base, uint32_t *status)
 {
+    grid_dep_wait();
     extern __shared__ int32_t s_cnt[];
     for (int e = threadIdx.x; e < N; e += kThreads)
         s_cnt[e] = 0;
@@ -72,6 +73,7 @@ __global__ void __launch_bounds__(1024)
                          int32_t *__restrict__ offsets, const float *__restrict__ p_mean,
                          float *__restrict__ f, float *__restrict__ aux_loss, float alpha)
 {
+    grid_dep_wait();
     __shared__ int32_t s_warp[32];
     __shared__ double s_aux[1024];
     const int e = threadIdx.x;
@@ -142,6 +144,7 @@ __global__ void __launch_bounds__(kThreads)
                          const int32_t *__restrict__ offsets, int32_t *__restrict__ perm,
                          int32_t *__restrict__ inv_row, uint8_t *__restrict__ drop)
 {
+    grid_dep_wait();
     extern __shared__ int32_t s_w[];  // [kWarps][N]
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     for (int i = threadIdx.x; i < kWarps * N; i += kThreads)
@@ -213,6 +216,7 @@ __global__ void __launch_bounds__(kThreads)
                            uint8_t *__restrict__ x_perm, float *__restrict__ x_scale,
                            __nv_bfloat16 *__restrict__ x_bf16_copy)
 {
+    grid_dep_wait();
     const int lane = threadIdx.x & 31;
     const int64_t R = *R_ptr;
     const int64_t nwarps = static_cast<int64_t>(gridDim.x) * kWarps;
@@ -289,6 +293,7 @@ __global__ void __launch_bounds__(kThreads)
     fp8_to_bf16_kernel(const uint8_t *__restrict__ q, int d, const int32_t *__restrict__ R_ptr,
                        __nv_bfloat16 *__restrict__ out)
 {
+    grid_dep_wait();
     const int lane = threadIdx.x & 31;
     const int64_t R = *R_ptr;
     const int64_t nwarps = static_cast<int64_t>(gridDim.x) * kWarps;
@@ -321,6 +326,7 @@ __global__ void __launch_bounds__(kThreads)
     quantize_tokens_kernel(const uint8_t *__restrict__ x, int64_t T, int d,
                            __nv_bfloat16 *__restrict__ xq, float *__restrict__ scale_out)
 {
+    grid_dep_wait();
     const int lane = threadIdx.x & 31;
     const int64_t nwarps = static_cast<int64_t>(gridDim.x) * kWarps;
     const int chunks = d / 8;
@@ -369,6 +375,7 @@ __global__ void __launch_bounds__(kThreads)
                             const int32_t *__restrict__ R_ptr, uint8_t *__restrict__ out,
                             float *__restrict__ out_scale)
 {
+    grid_dep_wait();
     const int lane = threadIdx.x & 31;
     const int64_t R = *R_ptr;
     const int64_t nwarps = static_cast<int64_t>(gridDim.x) * kWarps;
@@ -415,12 +422,12 @@ cudaError_t launch_dispatch(const DispatchLaunch &L, cudaStream_t stream)
     if (n_pairs == 0)
         return cudaSuccess;
     const int nblk = static_cast<int>((n_pairs + kDispChunk - 1) / kDispChunk);
-    dispatch_count_kernel<<<nblk, kThreads, L.N * sizeof(int32_t), stream>>>(
+    launch_k(dispatch_count_kernel, nblk, kThreads, L.N * sizeof(int32_t), stream, 
         L.topk_idx, n_pairs, L.N, L.block_base, L.status);
-    dispatch_scan_kernel<<<1, 1024, 0, stream>>>(nblk, L.N, n_pairs, L.capacity, L.block_base,
+    launch_k(dispatch_scan_kernel, 1, 1024, 0, stream, nblk, L.N, n_pairs, L.capacity, L.block_base,
                                                  L.counts, L.offsets, L.p_mean, L.f, L.aux_loss,
                                                  L.aux_alpha);
-    dispatch_rank_kernel<<<nblk, kThreads, kWarps * L.N * sizeof(int32_t), stream>>>(
+    launch_k(dispatch_rank_kernel, nblk, kThreads, kWarps * L.N * sizeof(int32_t), stream, 
         L.topk_idx, n_pairs, L.N, L.capacity, L.block_base, L.offsets, L.perm, L.inv_row, L.drop);
     if (L.x_perm == nullptr) {      // the caller builds the expert-ordered rows itself
         count_launches(3);
@@ -430,13 +437,13 @@ cudaError_t launch_dispatch(const DispatchLaunch &L, cudaStream_t stream)
     const uint8_t *x = static_cast<const uint8_t *>(L.x);
     uint8_t *xp = static_cast<uint8_t *>(L.x_perm);
     if (L.dtype == MOE_F32)
-        dispatch_gather_kernel<false, false><<<grid, kThreads, 0, stream>>>(
+        launch_k(dispatch_gather_kernel<false, false>, grid, kThreads, 0, stream, 
             x, L.d, L.k, L.perm, L.offsets + L.N, xp, nullptr, nullptr);
     else if (!L.fp8)
-        dispatch_gather_kernel<true, false><<<grid, kThreads, 0, stream>>>(
+        launch_k(dispatch_gather_kernel<true, false>, grid, kThreads, 0, stream, 
             x, L.d, L.k, L.perm, L.offsets + L.N, xp, nullptr, nullptr);
     else
-        dispatch_gather_kernel<true, true><<<grid, kThreads, 0, stream>>>(
+        launch_k(dispatch_gather_kernel<true, true>, grid, kThreads, 0, stream, 
             x, L.d, L.k, L.perm, L.offsets + L.N, xp, L.x_scale,
             static_cast<__nv_bfloat16 *>(L.x_bf16_copy));
     count_launches(4);
@@ -448,7 +455,7 @@ cudaError_t launch_quantize_tokens(const void *x, int64_t T, int32_t d, void *xq
 {
     if (T == 0)
         return cudaSuccess;
-    quantize_tokens_kernel<<<gather_grid(T), kThreads, 0, stream>>>(
+    launch_k(quantize_tokens_kernel, gather_grid(T), kThreads, 0, stream, 
         static_cast<const uint8_t *>(x), T, d, static_cast<__nv_bfloat16 *>(xq), scale);
     count_launches(1);
     return cudaGetLastError();
@@ -460,7 +467,7 @@ cudaError_t launch_gather_quantized(const void *xq, const float *scale, int64_t 
 {
     if (T == 0)
         return cudaSuccess;
-    gather_quantized_kernel<<<gather_grid(T * k), kThreads, 0, stream>>>(
+    launch_k(gather_quantized_kernel, gather_grid(T * k), kThreads, 0, stream, 
         static_cast<const uint8_t *>(xq), scale, d, k, perm, offsets + N,
         static_cast<uint8_t *>(out), out_scale);
     count_launches(1);
@@ -472,7 +479,7 @@ cudaError_t launch_fp8_to_bf16(const uint8_t *q, int64_t rows_cap, int32_t d,
 {
     if (rows_cap == 0)
         return cudaSuccess;
-    fp8_to_bf16_kernel<<<gather_grid(rows_cap), kThreads, 0, stream>>>(
+    launch_k(fp8_to_bf16_kernel, gather_grid(rows_cap), kThreads, 0, stream, 
         q, d, offsets + N, static_cast<__nv_bfloat16 *>(out));
     count_launches(1);
     return cudaGetLastError();

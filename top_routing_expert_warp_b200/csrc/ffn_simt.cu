@@ -22,6 +22,7 @@ __global__ void __launch_bounds__(kThreads)
                          const int32_t *__restrict__ offsets, int G, int rows_single,
                          float *__restrict__ out)
 {
+    grid_dep_wait();
     extern __shared__ float s_a[];
     int64_t R = offsets ? offsets[G] : rows_single;
     if (R > rows_cap)
@@ -82,13 +83,13 @@ cudaError_t launch_simt_gemm_f32(int epi, const float *A, int64_t rows_cap, int3
     if (smem > 48 * 1024)
         return cudaErrorInvalidValue;
     if (epi == EPI_SWIGLU)
-        simt_gemm_f32_kernel<EPI_SWIGLU><<<static_cast<int>(grid), kThreads, smem, stream>>>(
+        launch_k(simt_gemm_f32_kernel<EPI_SWIGLU>, static_cast<int>(grid), kThreads, smem, stream, 
             A, rows_cap, K, B, B2, n_out, offsets, G, rows_single, out);
     else if (epi == EPI_RELU)
-        simt_gemm_f32_kernel<EPI_RELU><<<static_cast<int>(grid), kThreads, smem, stream>>>(
+        launch_k(simt_gemm_f32_kernel<EPI_RELU>, static_cast<int>(grid), kThreads, smem, stream, 
             A, rows_cap, K, B, B2, n_out, offsets, G, rows_single, out);
     else
-        simt_gemm_f32_kernel<EPI_STORE><<<static_cast<int>(grid), kThreads, smem, stream>>>(
+        launch_k(simt_gemm_f32_kernel<EPI_STORE>, static_cast<int>(grid), kThreads, smem, stream, 
             A, rows_cap, K, B, B2, n_out, offsets, G, rows_single, out);
     count_launches(1);
     return cudaGetLastError();

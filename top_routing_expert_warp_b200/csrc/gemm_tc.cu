@@ -181,6 +181,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                     const __grid_constant__ CUtensorMap tmB, const __grid_constant__ CUtensorMap tmB2,
                     GemmParams p)
 {
+    grid_dep_wait();
     using Geo = Geometry<BN, EPI>;
     constexpr int STAGES = Geo::STAGES;
     constexpr int OUTN = Geo::OUTN;
@@ -627,8 +628,7 @@ cudaError_t launch_impl(const GemmLaunch &L, cudaStream_t stream)
     int grid = static_cast<int>(tiles_max < sm_count() ? tiles_max : sm_count());
     if (grid <= 0)
         return cudaSuccess;
-    grouped_gemm_tc<BN, EPI, OUT_F32>
-        <<<grid, kThreads, Geo::SMEM_BYTES, stream>>>(mA, mA16, mB, mB2, p);
+    launch_k(grouped_gemm_tc<BN, EPI, OUT_F32>, grid, kThreads, Geo::SMEM_BYTES, stream, mA, mA16, mB, mB2, p);
     count_launches(1);
     return cudaGetLastError();
 }
@@ -640,7 +640,8 @@ int router_ksplit(int64_t T, int32_t N, int32_t d)
     const int64_t m_tiles = (T + BM - 1) / BM;
     const int64_t KB = (d + BK - 1) / BK;
     (void)N;  // one n tile (N <= 256)
-    int64_t ks = (sm_count() + m_tiles - 1) / m_tiles;
+    // as many slices as keep the tiles within one wave of the SMs
+    int64_t ks = sm_count() / m_tiles;
     const int64_t cap = router_ksplit_cap(T, N);
     if (ks > cap)
         ks = cap;

@@ -3,9 +3,32 @@
 #pragma once
 
 #include <cstdint>
+#include <utility>
 #include <cuda_runtime.h>
 
 namespace moe {
+
+// Every kernel of the library is launched with programmatic dependent launch:
+// it may be scheduled while the previous kernel on the stream drains, and it
+// waits (griddepcontrol.wait, first thing in every kernel) until that kernel
+// has completed and its writes are visible.  This hides the launch gap
+// between the short kernels of a layer forward.
+template <typename... KArgs, typename... Args>
+inline cudaError_t launch_k(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem,
+                           cudaStream_t stream, Args &&...args)
+{
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = grid;
+    cfg.blockDim = block;
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = stream;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    return cudaLaunchKernelEx(&cfg, kernel, std::forward<Args>(args)...);
+}
 
 // Count of kernel launches made by the library (reported by moe_launch_count).
 void count_launches(int n);

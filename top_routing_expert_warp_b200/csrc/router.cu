@@ -184,6 +184,7 @@ __global__ void __launch_bounds__(kThreads)
                         int32_t *__restrict__ topk_idx, float *__restrict__ topk_w,
                         double *__restrict__ p_part)
 {
+    grid_dep_wait();
     __shared__ double s_p[kWarps][NMAX];
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int esz = BF16 ? 2 : 4;
@@ -317,6 +318,7 @@ __global__ void __launch_bounds__(kThreads, 2)
                          int32_t *__restrict__ topk_idx, float *__restrict__ topk_w,
                          double *__restrict__ p_part)
 {
+    grid_dep_wait();
     extern __shared__ double s_pdyn[];  // [kWarps][N]
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int chunks = d / 8;
@@ -411,9 +413,12 @@ __global__ void __launch_bounds__(kThreads, 2)
         double acc[KCM];
 #pragma unroll
         for (int c = 0; c < KCM; ++c) {
-            acc[c] = warp_sum(static_cast<double>(da[c].hi) + static_cast<double>(da[c].lo));
-            if (bias != nullptr && c < KC)
-                acc[c] += static_cast<double>(bias[cand[c]]);
+            acc[c] = 0.0;
+            if (c < KC) {   // KC is the same on every lane
+                acc[c] = warp_sum(static_cast<double>(da[c].hi) + static_cast<double>(da[c].lo));
+                if (bias != nullptr)
+                    acc[c] += static_cast<double>(bias[cand[c]]);
+            }
         }
         // order candidates by (recomputed value desc, index asc); fixed-shape
         // exchange sort so that every index is a compile-time constant
@@ -439,48 +444,57 @@ __global__ void __launch_bounds__(kThreads, 2)
         }
         const double mx = acc[0];
         const float mxf = static_cast<float>(mx);
-        // softmax denominator: candidates in fp64, the others in fp32
+        // candidates' exponentials in fp64, once per warp (every lane holds
+        // the same values); the other experts' in fp32 on their lanes
+        double ec[KCM];
+        double zc = 0.0, gs = 0.0;
+#pragma unroll
+        for (int c = 0; c < KCM; ++c) {
+            ec[c] = (c < KC) ? exp(acc[c] - mx) : 0.0;
+            zc += ec[c];
+            if (c < k)
+                gs += ec[c];
+        }
         float ev[NPL];
-        double zl = 0.0;
+        float zl = 0.0f;
 #pragma unroll
         for (int i = 0; i < NPL; ++i) {
             const int e = lane + 32 * i;
-            ev[i] = 0.0f;
-            if (e < N) {
-                double ce = -1.0;
+            bool is_c = false;
 #pragma unroll
-                for (int c = 0; c < KCM; ++c)
-                    if (c < KC && cand[c] == e)
-                        ce = exp(acc[c] - mx);
-                if (ce >= 0.0) {
-                    zl += ce;
-                    ev[i] = static_cast<float>(ce);
-                } else {
-                    ev[i] = expf(lv[i] - mxf);
-                    zl += static_cast<double>(ev[i]);
-                }
-            }
+            for (int c = 0; c < KCM; ++c)
+                is_c |= (c < KC && cand[c] == e);
+            ev[i] = (e < N && !is_c) ? expf(lv[i] - mxf) : 0.0f;
+            zl += ev[i];
         }
-        const double Z = warp_sum(zl);
-        const float zinv = static_cast<float>(1.0 / Z);
 #pragma unroll
-        for (int i = 0; i < NPL; ++i)
-            psum[i] += ev[i] * zinv;
-        // gates: lane j < k computes slot j from the recomputed logits
-        double aj = 0.0;
+        for (int o = 16; o > 0; o >>= 1)
+            zl += __shfl_xor_sync(0xffffffffu, zl, o);
+        const double Z = static_cast<double>(zl) + zc;
+        const double zinv = 1.0 / Z;
+#pragma unroll
+        for (int i = 0; i < NPL; ++i) {
+            const int e = lane + 32 * i;
+            float pv = ev[i] * static_cast<float>(zinv);
+#pragma unroll
+            for (int c = 0; c < KCM; ++c)
+                if (c < KC && cand[c] == e)
+                    pv = static_cast<float>(ec[c] * zinv);
+            psum[i] += pv;
+        }
+        // gates: slot j = the j-th recomputed candidate (lane j writes it)
+        double gj = 0.0;
         int ej = 0;
 #pragma unroll
         for (int c = 0; c < KCM; ++c)
             if (c == lane) {
-                aj = acc[c];
+                gj = ec[c];
                 ej = cand[c];
             }
-        double gj = (lane < k) ? exp(aj - mx) : 0.0;
-        const double gs = warp_sum(gj);
         const bool norm = (gate_mode == MOE_GATE_TOPK_THEN_SOFTMAX) || renorm;
         if (lane < k) {
             topk_idx[t * k + lane] = ej;
-            topk_w[t * k + lane] = static_cast<float>(norm ? gj / gs : gj / Z);
+            topk_w[t * k + lane] = static_cast<float>(norm ? gj / gs : gj * zinv);
         }
     }
 #pragma unroll
@@ -504,6 +518,7 @@ __global__ void __launch_bounds__(256)
     p_finalize_kernel(const double *__restrict__ p_part, int nblk, int N, int64_t T,
                       float *__restrict__ p_mean)
 {
+    grid_dep_wait();
     __shared__ double s[256];
     const int e = blockIdx.x;
     double acc = 0.0;
@@ -543,20 +558,20 @@ cudaError_t launch_router_small(RouterLaunch &L, cudaStream_t stream)
     *L.p_blocks = grid;
     if (L.dtype == MOE_BF16) {
         if (L.N <= 8)
-            router_small_kernel<true, 8><<<grid, kThreads, 0, stream>>>(
+            launch_k(router_small_kernel<true, 8>, grid, kThreads, 0, stream, 
                 L.x, L.Wg, L.bias, L.T, L.d, L.N, L.k, L.gate_mode, L.renormalize,
                 L.logits_out, L.topk_idx, L.topk_w, L.p_part);
         else
-            router_small_kernel<true, 16><<<grid, kThreads, 0, stream>>>(
+            launch_k(router_small_kernel<true, 16>, grid, kThreads, 0, stream, 
                 L.x, L.Wg, L.bias, L.T, L.d, L.N, L.k, L.gate_mode, L.renormalize,
                 L.logits_out, L.topk_idx, L.topk_w, L.p_part);
     } else {
         if (L.N <= 8)
-            router_small_kernel<false, 8><<<grid, kThreads, 0, stream>>>(
+            launch_k(router_small_kernel<false, 8>, grid, kThreads, 0, stream, 
                 L.x, L.Wg, L.bias, L.T, L.d, L.N, L.k, L.gate_mode, L.renormalize,
                 L.logits_out, L.topk_idx, L.topk_w, L.p_part);
         else
-            router_small_kernel<false, 16><<<grid, kThreads, 0, stream>>>(
+            launch_k(router_small_kernel<false, 16>, grid, kThreads, 0, stream, 
                 L.x, L.Wg, L.bias, L.T, L.d, L.N, L.k, L.gate_mode, L.renormalize,
                 L.logits_out, L.topk_idx, L.topk_w, L.p_part);
     }
@@ -567,7 +582,7 @@ cudaError_t launch_router_small(RouterLaunch &L, cudaStream_t stream)
 template <int NPL, int KCM>
 void select_launch(RouterLaunch &L, int grid, size_t smem, cudaStream_t stream)
 {
-    router_select_kernel<NPL, KCM><<<grid, kThreads, smem, stream>>>(
+    launch_k(router_select_kernel<NPL, KCM>, grid, kThreads, smem, stream, 
         L.logits_in, L.ksplit, L.logits_out, static_cast<const uint16_t *>(L.x),
         static_cast<const uint16_t *>(L.Wg), L.bias, L.T, L.d, L.N, L.k, L.gate_mode,
         L.renormalize, L.topk_idx, L.topk_w, L.p_part);
@@ -610,7 +625,7 @@ cudaError_t launch_router_select(RouterLaunch &L, cudaStream_t stream)
 cudaError_t launch_p_finalize(const double *p_part, int32_t p_blocks, int32_t N, int64_t T,
                               float *p_mean, cudaStream_t stream)
 {
-    p_finalize_kernel<<<N, 256, 0, stream>>>(p_part, p_blocks, N, T, p_mean);
+    launch_k(p_finalize_kernel, N, 256, 0, stream, p_part, p_blocks, N, T, p_mean);
     count_launches(1);
     return cudaGetLastError();
 }
