@@ -22,7 +22,9 @@ constexpr int kThreads = 256;
 constexpr int kWarps = kThreads / 32;
 constexpr int kMaxK = 8;
 
-template <bool BF16>
+// KM: bound on k (the loads of all slots are held in registers at once);
+// U chunks per lane per pass (4 for k <= 2, else 2).
+template <bool BF16, int KM>
 __global__ void __launch_bounds__(kThreads)
     combine_kernel(const uint8_t *__restrict__ y_perm, const int32_t *__restrict__ inv_row,
                    const float *__restrict__ topk_w, const uint8_t *__restrict__ y_shared,
@@ -36,8 +38,8 @@ __global__ void __launch_bounds__(kThreads)
     const int64_t nwarps = static_cast<int64_t>(gridDim.x) * kWarps;
     for (int64_t t = static_cast<int64_t>(blockIdx.x) * kWarps + (threadIdx.x >> 5); t < T;
          t += nwarps) {
-        int32_t row[kMaxK];
-        float g[kMaxK];
+        int32_t row[KM];
+        float g[KM];
         int32_t my_row = -1;
         float my_g = 0.0f;
         if (lane < k) {
@@ -49,19 +51,19 @@ __global__ void __launch_bounds__(kThreads)
             }
         }
 #pragma unroll
-        for (int j = 0; j < kMaxK; ++j) {
+        for (int j = 0; j < KM; ++j) {
             row[j] = __shfl_sync(0xffffffffu, my_row, j);
             g[j] = __shfl_sync(0xffffffffu, my_g, j);
         }
         // U chunks per lane per pass; the loads of every slot are issued
         // before any is used (predicated, no branches), so k * U loads per
         // lane are in flight at once
-        constexpr int U = 2;
+        constexpr int U = KM >= 4 ? 2 : 4;
         constexpr int V = BF16 ? 8 : 4;
         for (int c0 = lane; c0 < chunks; c0 += 32 * U) {
-            uint4 v[kMaxK][U];
+            uint4 v[KM][U];
 #pragma unroll
-            for (int j = 0; j < kMaxK; ++j) {
+            for (int j = 0; j < KM; ++j) {
                 const uint4 *src = reinterpret_cast<const uint4 *>(
                     y_perm + static_cast<int64_t>(row[j] > 0 ? row[j] : 0) * d * esz);
 #pragma unroll
@@ -78,7 +80,7 @@ __global__ void __launch_bounds__(kThreads)
                 for (int i = 0; i < V; ++i)
                     acc[u][i] = 0.0f;
 #pragma unroll
-            for (int j = 0; j < kMaxK; ++j) {
+            for (int j = 0; j < KM; ++j) {
                 if (j < k && row[j] >= 0) {
 #pragma unroll
                     for (int u = 0; u < U; ++u) {
@@ -152,16 +154,27 @@ cudaError_t launch_combine(int dtype, const void *y_perm, const int32_t *inv_row
     if (grid > static_cast<int64_t>(sms) * 8)
         grid = static_cast<int64_t>(sms) * 8;
     const int64_t rows_cap = T * k;
-    if (dtype == MOE_BF16)
-        launch_k(combine_kernel<true>, static_cast<int>(grid), kThreads, 0, stream, 
-            static_cast<const uint8_t *>(y_perm), inv_row, topk_w,
-            static_cast<const uint8_t *>(y_shared), static_cast<uint8_t *>(y), T, d, k, rows_cap,
-            status);
-    else
-        launch_k(combine_kernel<false>, static_cast<int>(grid), kThreads, 0, stream, 
-            static_cast<const uint8_t *>(y_perm), inv_row, topk_w,
-            static_cast<const uint8_t *>(y_shared), static_cast<uint8_t *>(y), T, d, k, rows_cap,
-            status);
+    const uint8_t *yp = static_cast<const uint8_t *>(y_perm);
+    const uint8_t *ys = static_cast<const uint8_t *>(y_shared);
+    uint8_t *yo = static_cast<uint8_t *>(y);
+    const int g = static_cast<int>(grid);
+    if (dtype == MOE_BF16) {
+        if (k <= 1)
+            launch_k(combine_kernel<true, 1>, g, kThreads, 0, stream, yp, inv_row, topk_w, ys, yo,
+                     T, d, k, rows_cap, status);
+        else if (k <= 2)
+            launch_k(combine_kernel<true, 2>, g, kThreads, 0, stream, yp, inv_row, topk_w, ys, yo,
+                     T, d, k, rows_cap, status);
+        else if (k <= 4)
+            launch_k(combine_kernel<true, 4>, g, kThreads, 0, stream, yp, inv_row, topk_w, ys, yo,
+                     T, d, k, rows_cap, status);
+        else
+            launch_k(combine_kernel<true, kMaxK>, g, kThreads, 0, stream, yp, inv_row, topk_w, ys,
+                     yo, T, d, k, rows_cap, status);
+    } else {
+        launch_k(combine_kernel<false, kMaxK>, g, kThreads, 0, stream, yp, inv_row, topk_w, ys, yo,
+                 T, d, k, rows_cap, status);
+    }
     count_launches(1);
     return cudaGetLastError();
 }

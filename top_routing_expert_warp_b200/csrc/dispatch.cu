@@ -67,26 +67,23 @@ __global__ void __launch_bounds__(kThreads)
         block_base[static_cast<int64_t>(blockIdx.x) * N + e] = s_cnt[e];
 }
 
-__global__ void __launch_bounds__(1024)
-    dispatch_scan_kernel(int nblk, int N, int64_t n_pairs, int64_t C,
-                         int32_t *__restrict__ block_base, int32_t *__restrict__ counts,
-                         int32_t *__restrict__ offsets, const float *__restrict__ p_mean,
-                         float *__restrict__ f, float *__restrict__ aux_loss, float alpha)
+// Per expert e (thread e of a 1024-thread block, e < N): total count `run`,
+// kept = min(run, C), offsets = exclusive scan of kept over experts, f and
+// L_aux = alpha N sum_e f_e p_e summed in a fixed tree order.  Also leaves
+// offsets in s_off when it is given.  Every thread of the block calls it.
+__device__ __forceinline__ void expert_offsets_and_aux(int e, int32_t run, int N, int64_t n_pairs,
+                                                       int64_t C, int32_t *__restrict__ counts,
+                                                       int32_t *__restrict__ offsets,
+                                                       const float *__restrict__ p_mean,
+                                                       float *__restrict__ f,
+                                                       float *__restrict__ aux_loss, float alpha,
+                                                       int32_t *s_off)
 {
-    grid_dep_wait();
     __shared__ int32_t s_warp[32];
     __shared__ double s_aux[1024];
-    const int e = threadIdx.x;
     const int lane = e & 31, warp = e >> 5;
     int32_t kept = 0;
-    int32_t run = 0;
     if (e < N) {
-        for (int b = 0; b < nblk; ++b) {
-            const int64_t o = static_cast<int64_t>(b) * N + e;
-            const int32_t v = block_base[o];
-            block_base[o] = run;
-            run += v;
-        }
         counts[e] = run;
         kept = (C >= 0 && run > C) ? static_cast<int32_t>(C) : run;
         if (f != nullptr)
@@ -116,8 +113,11 @@ __global__ void __launch_bounds__(1024)
     }
     __syncthreads();
     const int32_t excl = s_warp[warp] + incl - kept;
-    if (e < N)
+    if (e < N) {
         offsets[e] = excl;
+        if (s_off != nullptr)
+            s_off[e] = excl;
+    }
     if (e == N - 1)
         offsets[N] = excl + kept;
     // L_aux = alpha N sum_e f_e p_e, summed in a fixed tree order
@@ -128,13 +128,131 @@ __global__ void __launch_bounds__(1024)
                    static_cast<double>(p_mean[e]);
         s_aux[e] = term;
         __syncthreads();
-        for (int s = 512; s > 0; s >>= 1) {
-            if (e < s)
-                s_aux[e] += s_aux[e + s];
+        for (int st = 512; st > 0; st >>= 1) {
+            if (e < st)
+                s_aux[e] += s_aux[e + st];
             __syncthreads();
         }
         if (e == 0)
             *aux_loss = static_cast<float>(static_cast<double>(alpha) * N * s_aux[0]);
+    }
+}
+
+__global__ void __launch_bounds__(1024)
+    dispatch_scan_kernel(int nblk, int N, int64_t n_pairs, int64_t C,
+                         int32_t *__restrict__ block_base, int32_t *__restrict__ counts,
+                         int32_t *__restrict__ offsets, const float *__restrict__ p_mean,
+                         float *__restrict__ f, float *__restrict__ aux_loss, float alpha)
+{
+    grid_dep_wait();
+    const int e = threadIdx.x;
+    int32_t run = 0;
+    if (e < N) {
+        for (int b = 0; b < nblk; ++b) {
+            const int64_t o = static_cast<int64_t>(b) * N + e;
+            const int32_t v = block_base[o];
+            block_base[o] = run;
+            run += v;
+        }
+    }
+    expert_offsets_and_aux(e, run, N, n_pairs, C, counts, offsets, p_mean, f, aux_loss, alpha,
+                           nullptr);
+}
+
+// The whole sort in one block, for batches of at most kFusedMaxPairs pairs and
+// N <= kFusedMaxN experts: each of the 32 warps takes a contiguous range of
+// pairs (in pair order), counts its experts, a column scan over the warps
+// gives every warp its base inside each expert, and a second walk over the
+// range (expert ids kept in shared memory) ranks each pair stably.  Same
+// results as count + scan + rank, in one launch without a workspace.
+constexpr int kFusedThreads = 1024;
+constexpr int kFusedWarps = kFusedThreads / 32;
+
+__global__ void __launch_bounds__(kFusedThreads)
+    dispatch_fused_kernel(const int32_t *__restrict__ idx, int64_t n_pairs, int N, int64_t C,
+                          int32_t *__restrict__ counts, int32_t *__restrict__ offsets,
+                          int32_t *__restrict__ perm, int32_t *__restrict__ inv_row,
+                          uint8_t *__restrict__ drop, const float *__restrict__ p_mean,
+                          float *__restrict__ f, float *__restrict__ aux_loss, float alpha,
+                          uint32_t *status)
+{
+    grid_dep_wait();
+    extern __shared__ int32_t s_fz[];
+    int32_t *s_cnt = s_fz;                                              // [32][N]
+    int16_t *s_e = reinterpret_cast<int16_t *>(s_fz + kFusedWarps * N);  // [n_pairs]
+    __shared__ int32_t s_off[kFusedMaxN];
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    for (int i = threadIdx.x; i < kFusedWarps * N; i += kFusedThreads)
+        s_cnt[i] = 0;
+    __syncthreads();
+    // pairs per warp, a multiple of 32
+    const int64_t per_w = (n_pairs + 32 * kFusedWarps - 1) / (32 * kFusedWarps) * 32;
+    const int64_t wb = warp * per_w;
+    int32_t *mine = s_cnt + warp * N;
+    constexpr int U = 4;   // rounds whose loads are issued together
+    for (int64_t r0 = 0; r0 < per_w; r0 += 32 * U) {
+        int ev[U];
+#pragma unroll
+        for (int u = 0; u < U; ++u) {
+            const int64_t i = wb + r0 + 32 * u + lane;
+            ev[u] = (r0 + 32 * u < per_w && i < n_pairs) ? idx[i] : -1;
+        }
+#pragma unroll
+        for (int u = 0; u < U; ++u) {
+            if (r0 + 32 * u >= per_w)
+                break;
+            const int64_t i = wb + r0 + 32 * u + lane;
+            int e = ev[u];
+            if (i < n_pairs) {
+                if (e < 0 || e >= N) {
+                    set_status(status, DEV_BAD_EXPERT);
+                    e = -1;
+                }
+                s_e[i] = static_cast<int16_t>(e);
+            }
+            const uint32_t peers = __match_any_sync(0xffffffffu, e);
+            if (e >= 0 && lane == __ffs(peers) - 1)
+                mine[e] += __popc(peers);
+            __syncwarp();
+        }
+    }
+    __syncthreads();
+    // column scan: warp w's base inside expert e = pairs of e in warps < w
+    int32_t run = 0;
+    if (threadIdx.x < N) {
+        const int e = threadIdx.x;
+        for (int w = 0; w < kFusedWarps; ++w) {
+            const int32_t v = s_cnt[w * N + e];
+            s_cnt[w * N + e] = run;
+            run += v;
+        }
+    }
+    expert_offsets_and_aux(threadIdx.x, run, N, n_pairs, C, counts, offsets, p_mean, f, aux_loss,
+                           alpha, s_off);
+    __syncthreads();
+    // walk again in order; rank = warp base + earlier rounds + earlier lanes
+    for (int64_t r = 0; r < per_w; r += 32) {
+        const int64_t i = wb + r + lane;
+        const int e = i < n_pairs ? static_cast<int>(s_e[i]) : -1;
+        const uint32_t peers = __match_any_sync(0xffffffffu, e);
+        int32_t rank = 0;
+        if (e >= 0)
+            rank = mine[e] + __popc(peers & lanemask_lt());
+        __syncwarp();
+        if (e >= 0 && lane == __ffs(peers) - 1)
+            mine[e] += __popc(peers);
+        __syncwarp();
+        if (i < n_pairs) {
+            if (e < 0 || (C >= 0 && rank >= C)) {
+                drop[i] = 1;
+                inv_row[i] = -1;
+            } else {
+                const int32_t row = s_off[e] + rank;
+                perm[row] = static_cast<int32_t>(i);
+                inv_row[i] = row;
+                drop[i] = 0;
+            }
+        }
     }
 }
 
@@ -421,16 +539,36 @@ cudaError_t launch_dispatch(const DispatchLaunch &L, cudaStream_t stream)
     const int64_t n_pairs = L.T * L.k;
     if (n_pairs == 0)
         return cudaSuccess;
-    const int nblk = static_cast<int>((n_pairs + kDispChunk - 1) / kDispChunk);
-    launch_k(dispatch_count_kernel, nblk, kThreads, L.N * sizeof(int32_t), stream, 
-        L.topk_idx, n_pairs, L.N, L.block_base, L.status);
-    launch_k(dispatch_scan_kernel, 1, 1024, 0, stream, nblk, L.N, n_pairs, L.capacity, L.block_base,
-                                                 L.counts, L.offsets, L.p_mean, L.f, L.aux_loss,
-                                                 L.aux_alpha);
-    launch_k(dispatch_rank_kernel, nblk, kThreads, kWarps * L.N * sizeof(int32_t), stream, 
-        L.topk_idx, n_pairs, L.N, L.capacity, L.block_base, L.offsets, L.perm, L.inv_row, L.drop);
+    int sort_launches;
+    if (n_pairs <= kFusedMaxPairs && L.N <= kFusedMaxN) {
+        const size_t smem = kFusedWarps * L.N * sizeof(int32_t) + n_pairs * sizeof(int16_t);
+        static bool attr_set = false;   // one size bound for every device and call
+        if (!attr_set) {
+            const cudaError_t err = cudaFuncSetAttribute(
+                dispatch_fused_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                static_cast<int>(kFusedWarps * kFusedMaxN * sizeof(int32_t) +
+                                 kFusedMaxPairs * sizeof(int16_t)));
+            if (err != cudaSuccess)
+                return err;
+            attr_set = true;
+        }
+        launch_k(dispatch_fused_kernel, 1, kFusedThreads, smem, stream, L.topk_idx, n_pairs, L.N,
+                 L.capacity, L.counts, L.offsets, L.perm, L.inv_row, L.drop, L.p_mean, L.f,
+                 L.aux_loss, L.aux_alpha, L.status);
+        sort_launches = 1;
+    } else {
+        const int nblk = static_cast<int>((n_pairs + kDispChunk - 1) / kDispChunk);
+        launch_k(dispatch_count_kernel, nblk, kThreads, L.N * sizeof(int32_t), stream,
+                 L.topk_idx, n_pairs, L.N, L.block_base, L.status);
+        launch_k(dispatch_scan_kernel, 1, 1024, 0, stream, nblk, L.N, n_pairs, L.capacity,
+                 L.block_base, L.counts, L.offsets, L.p_mean, L.f, L.aux_loss, L.aux_alpha);
+        launch_k(dispatch_rank_kernel, nblk, kThreads, kWarps * L.N * sizeof(int32_t), stream,
+                 L.topk_idx, n_pairs, L.N, L.capacity, L.block_base, L.offsets, L.perm,
+                 L.inv_row, L.drop);
+        sort_launches = 3;
+    }
     if (L.x_perm == nullptr) {      // the caller builds the expert-ordered rows itself
-        count_launches(3);
+        count_launches(sort_launches);
         return cudaGetLastError();
     }
     const int grid = gather_grid(n_pairs);
@@ -446,7 +584,7 @@ cudaError_t launch_dispatch(const DispatchLaunch &L, cudaStream_t stream)
         launch_k(dispatch_gather_kernel<true, true>, grid, kThreads, 0, stream, 
             x, L.d, L.k, L.perm, L.offsets + L.N, xp, L.x_scale,
             static_cast<__nv_bfloat16 *>(L.x_bf16_copy));
-    count_launches(4);
+    count_launches(sort_launches + 1);
     return cudaGetLastError();
 }
 

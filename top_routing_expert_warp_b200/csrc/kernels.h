@@ -114,6 +114,10 @@ cudaError_t launch_p_finalize(const double *p_part, int32_t p_blocks, int32_t N,
 
 // Dispatch: see dispatch.cu.
 constexpr int kDispChunk = 2048;      // (token, slot) pairs per block
+// Batches of at most kFusedMaxPairs pairs over at most kFusedMaxN experts are
+// sorted by one block in one launch (expert ids staged in shared memory).
+constexpr int64_t kFusedMaxPairs = 8192;
+constexpr int kFusedMaxN = 256;
 struct DispatchLaunch {
     int dtype;                // element type of x
     int fp8;                  // quantise rows to E4M3 + per-row scale

@@ -266,10 +266,12 @@ __global__ void __launch_bounds__(kThreads)
     }
 }
 
-// (value, index) ordering: larger value first, then lower index.
-__device__ __forceinline__ bool better(float v1, int e1, float v2, int e2)
+// Unsigned key with the order of the float values (-0 counts as +0, so that
+// equal values get equal keys): larger key = larger value.
+__device__ __forceinline__ uint32_t order_key(float v)
 {
-    return (v1 > v2) || (v1 == v2 && e1 < e2 && e1 >= 0) || (e2 < 0 && e1 >= 0);
+    const uint32_t u = __float_as_uint(v + 0.0f);
+    return (u & 0x80000000u) ? ~u : (u | 0x80000000u);
 }
 
 // Compensated fp32 accumulator (hi + lo) of bf16 dot products; see DotAcc.
@@ -310,7 +312,7 @@ constexpr int kSelUnroll = 2;
 // Both are compile-time so that every loop below has a fixed trip count and
 // the instantiation used by a layer stays small.
 template <int NPL, int KCM>
-__global__ void __launch_bounds__(kThreads, 2)
+__global__ void __launch_bounds__(kThreads, NPL >= 8 ? 2 : 3)
     router_select_kernel(const float *__restrict__ part, int ksplit,
                          float *__restrict__ logits_out, const uint16_t *__restrict__ x,
                          const uint16_t *__restrict__ w, const float *__restrict__ bias, int64_t T,
@@ -355,7 +357,10 @@ __global__ void __launch_bounds__(kThreads, 2)
                 lv[i] = v;
             }
         }
-        // candidates: the KC best logits, best first
+        // candidates: the KC best logits, best first.  Each round takes the
+        // lane's best untaken logit (lowest index on a tie), then the warp's
+        // largest (two warp reductions: the largest value, then the lowest
+        // expert index holding it)
         int cand[KCM];
         uint32_t taken = 0;
 #pragma unroll
@@ -372,15 +377,10 @@ __global__ void __launch_bounds__(kThreads, 2)
                         be = e;
                     }
                 }
-#pragma unroll
-                for (int o = 16; o > 0; o >>= 1) {
-                    const float ov = __shfl_xor_sync(0xffffffffu, bv, o);
-                    const int oe = __shfl_xor_sync(0xffffffffu, be, o);
-                    if (better(ov, oe, bv, be)) {
-                        bv = ov;
-                        be = oe;
-                    }
-                }
+                const uint32_t key = be >= 0 ? order_key(bv) : 0u;
+                const uint32_t top = __reduce_max_sync(0xffffffffu, key);
+                be = static_cast<int>(__reduce_min_sync(
+                    0xffffffffu, (be >= 0 && key == top) ? static_cast<uint32_t>(be) : 0xffffffffu));
                 cand[c] = be;
                 if ((be & 31) == lane)
                     taken |= 1u << (be >> 5);
@@ -444,13 +444,19 @@ __global__ void __launch_bounds__(kThreads, 2)
         }
         const double mx = acc[0];
         const float mxf = static_cast<float>(mx);
-        // candidates' exponentials in fp64, once per warp (every lane holds
-        // the same values); the other experts' in fp32 on their lanes
+        // candidates' exponentials in fp64, candidate c on lane c, then
+        // broadcast; the other experts' in fp32 on their lanes
+        double my_acc = 0.0;
+#pragma unroll
+        for (int c = 0; c < KCM; ++c)
+            if (c == lane)
+                my_acc = acc[c];
+        const double my_ec = (lane < KC) ? exp(my_acc - mx) : 0.0;
         double ec[KCM];
         double zc = 0.0, gs = 0.0;
 #pragma unroll
         for (int c = 0; c < KCM; ++c) {
-            ec[c] = (c < KC) ? exp(acc[c] - mx) : 0.0;
+            ec[c] = (c < KC) ? __shfl_sync(0xffffffffu, my_ec, c) : 0.0;
             zc += ec[c];
             if (c < k)
                 gs += ec[c];
