@@ -138,3 +138,38 @@ def test_pair_tiles_shared_expert():
     wl = synth.Workload("pair-shared", T=1100, d=256, N=4, k=1, H=128, act="swiglu",
                         dtype="bf16", gate_mode="F", renormalize=True, H_shared=256, seed=27)
     _layer_vs_oracle(wl)
+
+
+@pytest.mark.parametrize("act", ["swiglu", "relu"])
+def test_pair_tile_remainders(act):
+    # CTA-pair GEMM (>= 512 rows per expert on average) with each expert's
+    # last 256-row tile holding 1, 32, 33, 224 or 225 rows, or none (rows past
+    # the expert's segment belong to the next expert or lie past the array and
+    # must not reach the output); H = 384 leaves a partial column tile for ReLU
+    counts = np.array([513, 544, 545, 736, 737, 512])
+    wl = synth.Workload("pair-rem", T=int(counts.sum()), d=256, N=len(counts), k=1, H=384,
+                        act=act, dtype="bf16", gate_mode="R", seed=28)
+    assert wl.T >= 512 * wl.N
+    dev, host = upload_inputs(wl)
+    cfg = cfg_of(wl)
+    ws = moe.workspace(cfg)
+    offsets = np.concatenate([[0], np.cumsum(counts)]).astype(np.int32)
+    yp = torch.zeros((wl.T, wl.d), dtype=torch.bfloat16, device="cuda")
+    moe.moe_expert_ffn(cfg, dev["x"], None, torch.from_numpy(offsets).cuda(), dev["W1"],
+                       dev.get("W3"), dev["W2"], yp, ws)
+    assert moe.moe_check_status(ws)[0] == moe.MOE_OK
+    got = to_f64(yp)
+    xin = oracle.decode(host["x"])
+    exp_of_row = np.repeat(np.arange(wl.N), counts)
+    want = np.empty((wl.T, wl.d))
+    for r in range(wl.T):
+        e = exp_of_row[r]
+        want[r] = oracle.ffn_row(xin[r], host["W1"][e], host["W3"][e] if act == "swiglu" else None,
+                                 host["W2"][e], act)
+    # every expert's rows, the last tile's in particular, on their own
+    for e in range(wl.N):
+        lo, hi = offsets[e], offsets[e + 1]
+        tail = lo + (counts[e] // 256) * 256
+        assert rel_l2(got[lo:hi], want[lo:hi]) <= 5e-3, (e, "all rows")
+        if hi > tail:
+            assert rel_l2(got[tail:hi], want[tail:hi]) <= 5e-3, (e, "last tile")
