@@ -436,13 +436,17 @@ __global__ void __launch_bounds__(kThreads)
     }
 }
 
-// Per-token FP8 payload for the fused layer path: scale = amax / 448 (1 for
-// an all-zero row) and code = E4M3(x / scale) as in the gather kernel above;
-// writes the codes' values as bf16 (exact) for the expert GEMM, which gathers
-// token rows directly, and the per-token scale for its epilogue.
+// FP8 payload of the fused layer path, written straight into the expert-
+// ordered GEMM rows: one warp per token computes scale = amax / 448 (1 for an
+// all-zero row) and codes = E4M3(x / scale), as the gather kernel above does
+// per row, and writes the codes' values as bf16 (exact) to every kept row of
+// the token (inv_row), with the scale beside each row for the GEMM epilogue.
+// Each token is read twice from L2 and quantised once.
+template <int KM>
 __global__ void __launch_bounds__(kThreads)
-    quantize_tokens_kernel(const uint8_t *__restrict__ x, int64_t T, int d,
-                           __nv_bfloat16 *__restrict__ xq, float *__restrict__ scale_out)
+    quantize_scatter_kernel(const uint8_t *__restrict__ x, int64_t T, int d, int k,
+                            const int32_t *__restrict__ inv_row, uint8_t *__restrict__ out,
+                            float *__restrict__ out_scale)
 {
     grid_dep_wait();
     const int lane = threadIdx.x & 31;
@@ -450,6 +454,11 @@ __global__ void __launch_bounds__(kThreads)
     const int chunks = d / 8;
     for (int64_t t = static_cast<int64_t>(blockIdx.x) * kWarps + (threadIdx.x >> 5); t < T;
          t += nwarps) {
+        int32_t rows[KM];
+        const int32_t my_row = lane < k ? inv_row[t * k + lane] : -1;
+#pragma unroll
+        for (int j = 0; j < KM; ++j)
+            rows[j] = __shfl_sync(0xffffffffu, my_row, j);
         const uint4 *src = reinterpret_cast<const uint4 *>(x + t * static_cast<int64_t>(d) * 2);
         float amax = 0.0f;
         for (int c = lane; c < chunks; c += 32) {
@@ -465,9 +474,8 @@ __global__ void __launch_bounds__(kThreads)
         for (int o = 16; o > 0; o >>= 1)
             amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, o));
         const float scale = amax > 0.0f ? __fdiv_rn(amax, 448.0f) : 1.0f;
-        if (lane == 0)
-            scale_out[t] = scale;
-        uint4 *dst = reinterpret_cast<uint4 *>(xq + t * static_cast<int64_t>(d));
+        if (lane < k && my_row >= 0)
+            out_scale[my_row] = scale;
         for (int c = lane; c < chunks; c += 32) {
             const uint4 v = __ldg(src + c);
             const uint32_t w[4] = {v.x, v.y, v.z, v.w};
@@ -481,41 +489,11 @@ __global__ void __launch_bounds__(kThreads)
                                                __NV_SATFINITE, __NV_E4M3);
                 b[i] = pack_bf16x2(static_cast<float>(lo), static_cast<float>(hi));
             }
-            dst[c] = make_uint4(b[0], b[1], b[2], b[3]);
-        }
-    }
-}
-
-// Expert-ordered bf16 rows and row scales from the per-token FP8 payload.
-__global__ void __launch_bounds__(kThreads)
-    gather_quantized_kernel(const uint8_t *__restrict__ xq, const float *__restrict__ scale,
-                            int d, int k, const int32_t *__restrict__ perm,
-                            const int32_t *__restrict__ R_ptr, uint8_t *__restrict__ out,
-                            float *__restrict__ out_scale)
-{
-    grid_dep_wait();
-    const int lane = threadIdx.x & 31;
-    const int64_t R = *R_ptr;
-    const int64_t nwarps = static_cast<int64_t>(gridDim.x) * kWarps;
-    const int chunks = d / 8;
-    for (int64_t r = static_cast<int64_t>(blockIdx.x) * kWarps + (threadIdx.x >> 5); r < R;
-         r += nwarps) {
-        const int64_t t = perm[r] / k;
-        if (lane == 0)
-            out_scale[r] = scale[t];
-        const uint4 *src = reinterpret_cast<const uint4 *>(xq + t * static_cast<int64_t>(d) * 2);
-        uint4 *dst = reinterpret_cast<uint4 *>(out + r * static_cast<int64_t>(d) * 2);
-        constexpr int U = 4;
-        for (int c0 = lane; c0 < chunks; c0 += 32 * U) {
-            uint4 v[U];
+            const uint4 o = make_uint4(b[0], b[1], b[2], b[3]);
 #pragma unroll
-            for (int u = 0; u < U; ++u)
-                if (c0 + 32 * u < chunks)
-                    v[u] = __ldg(src + c0 + 32 * u);
-#pragma unroll
-            for (int u = 0; u < U; ++u)
-                if (c0 + 32 * u < chunks)
-                    dst[c0 + 32 * u] = v[u];
+            for (int j = 0; j < KM; ++j)
+                if (j < k && rows[j] >= 0)
+                    reinterpret_cast<uint4 *>(out + static_cast<int64_t>(rows[j]) * d * 2)[c] = o;
         }
     }
 }
@@ -588,26 +566,23 @@ cudaError_t launch_dispatch(const DispatchLaunch &L, cudaStream_t stream)
     return cudaGetLastError();
 }
 
-cudaError_t launch_quantize_tokens(const void *x, int64_t T, int32_t d, void *xq, float *scale,
-                                   cudaStream_t stream)
+cudaError_t launch_quantize_scatter(const void *x, int64_t T, int32_t d, int32_t k,
+                                    const int32_t *inv_row, void *out, float *out_scale,
+                                    cudaStream_t stream)
 {
     if (T == 0)
         return cudaSuccess;
-    launch_k(quantize_tokens_kernel, gather_grid(T), kThreads, 0, stream, 
-        static_cast<const uint8_t *>(x), T, d, static_cast<__nv_bfloat16 *>(xq), scale);
-    count_launches(1);
-    return cudaGetLastError();
-}
-
-cudaError_t launch_gather_quantized(const void *xq, const float *scale, int64_t T, int32_t d,
-                                    int32_t k, const int32_t *perm, const int32_t *offsets,
-                                    int32_t N, void *out, float *out_scale, cudaStream_t stream)
-{
-    if (T == 0)
-        return cudaSuccess;
-    launch_k(gather_quantized_kernel, gather_grid(T * k), kThreads, 0, stream, 
-        static_cast<const uint8_t *>(xq), scale, d, k, perm, offsets + N,
-        static_cast<uint8_t *>(out), out_scale);
+    if (k < 1 || k > 8)
+        return cudaErrorInvalidValue;
+    const uint8_t *xs = static_cast<const uint8_t *>(x);
+    uint8_t *o = static_cast<uint8_t *>(out);
+    const int grid = gather_grid(T);
+    if (k <= 2)
+        launch_k(quantize_scatter_kernel<2>, grid, kThreads, 0, stream, xs, T, d, k, inv_row, o,
+                 out_scale);
+    else
+        launch_k(quantize_scatter_kernel<8>, grid, kThreads, 0, stream, xs, T, d, k, inv_row, o,
+                 out_scale);
     count_launches(1);
     return cudaGetLastError();
 }

@@ -142,14 +142,11 @@ struct DispatchLaunch {
     uint32_t *status;
 };
 cudaError_t launch_dispatch(const DispatchLaunch &L, cudaStream_t stream);
-// Per-token FP8 payload: scale[t] = amax/448, xq[t] = E4M3 codes of x[t]/scale as bf16.
-cudaError_t launch_quantize_tokens(const void *x, int64_t T, int32_t d, void *xq, float *scale,
-                                   cudaStream_t stream);
-// Rows < offsets[N] of the expert-ordered GEMM operand from the per-token
-// payload: out[r] = xq[perm[r] / k] (bf16), out_scale[r] = scale[perm[r] / k].
-cudaError_t launch_gather_quantized(const void *xq, const float *scale, int64_t T, int32_t d,
-                                    int32_t k, const int32_t *perm, const int32_t *offsets,
-                                    int32_t N, void *out, float *out_scale, cudaStream_t stream);
+// FP8 payload of token t written to every kept row r = inv_row[t k + j]:
+// out[r] = E4M3 codes of x[t] / scale as bf16, out_scale[r] = scale = amax/448.
+cudaError_t launch_quantize_scatter(const void *x, int64_t T, int32_t d, int32_t k,
+                                    const int32_t *inv_row, void *out, float *out_scale,
+                                    cudaStream_t stream);
 // E4M3 codes -> bf16 (exact) for rows < offsets[N].
 cudaError_t launch_fp8_to_bf16(const uint8_t *q, int64_t rows_cap, int32_t d,
                                const int32_t *offsets, int32_t N, void *out, cudaStream_t stream);

@@ -62,7 +62,7 @@ bool aligned(const void *p, size_t a) { return (reinterpret_cast<uintptr_t>(p) %
 // Offsets of the workspace regions (bytes from the workspace start).
 struct Layout {
     size_t status, p_part, logits, topk_idx, topk_w, p_mean, counts, offsets, block_base, perm,
-        inv_row, drop, x_scale, xq, tscale, x_gemm, h, y_perm, hs, ys, total;
+        inv_row, drop, x_scale, x_gemm, h, y_perm, hs, ys, total;
 };
 
 bool config_ok(const moe_config *c)
@@ -124,8 +124,6 @@ Layout layout_of(const moe_config &c)
     L.drop = take(rows);
     L.x_scale = take(rows * 4);
     const bool fp8 = c.dispatch_dtype == MOE_FP8_E4M3;
-    L.xq = take(fp8 ? T * d * 2 : 0);          // per-token FP8 payload as bf16 (fused path)
-    L.tscale = take(fp8 ? T * 4 : 0);          // its per-token scale
     L.x_gemm = take(rows * d * (fp8 ? 2 : static_cast<size_t>(elem_size(c.dtype))));  // GEMM rows
     L.h = take(rows * H * es);
     L.y_perm = take(rows * d * es);
@@ -482,19 +480,16 @@ moe_status moe_layer_forward(const moe_config *cfg, const void *x, const void *W
     prof_mark(1, s);
     // dispatch: counts, capacity, permutation, then the expert-ordered GEMM
     // rows.  FP8 dispatch quantises each token once (codes as bf16 + scale)
-    // and copies those rows, instead of quantising every (token, slot) copy.
+    // and writes them to the token's kept rows, instead of quantising every
+    // (token, slot) copy.
     void *xg = w.at<void>(w.L.x_gemm);
-    if (fp8 && c.T > 0)
-        MOE_CUDA(moe::launch_quantize_tokens(x, c.T, c.d, w.at<void>(w.L.xq),
-                                             w.at<float>(w.L.tscale), s));
     st = run_dispatch(c, x, idx, counts, offsets, w.at<int32_t>(w.L.perm),
                       w.at<int32_t>(w.L.inv_row), w.at<uint8_t>(w.L.drop), fp8 ? nullptr : xg,
                       nullptr, nullptr, pm, f, aux_loss, w, s);
     if (st != MOE_OK)
         return st;
     if (fp8 && c.T > 0)
-        MOE_CUDA(moe::launch_gather_quantized(w.at<void>(w.L.xq), w.at<float>(w.L.tscale), c.T,
-                                              c.d, c.k, w.at<int32_t>(w.L.perm), offsets, c.N, xg,
+        MOE_CUDA(moe::launch_quantize_scatter(x, c.T, c.d, c.k, w.at<int32_t>(w.L.inv_row), xg,
                                               w.at<float>(w.L.x_scale), s));
     prof_mark(2, s);
     if (c.T == 0) {
