@@ -173,3 +173,45 @@ def test_pair_tile_remainders(act):
         assert rel_l2(got[lo:hi], want[lo:hi]) <= 5e-3, (e, "all rows")
         if hi > tail:
             assert rel_l2(got[tail:hi], want[tail:hi]) <= 5e-3, (e, "last tile")
+
+
+@pytest.mark.parametrize("act,fp8", [("swiglu", False), ("relu", False), ("swiglu", True)])
+def test_gemm_combined_tiles(act, fp8):
+    # one-CTA GEMM (< 512 rows per expert on average): experts a few rows past
+    # 128 or 256 (129, 150, 176, 304) put those rows in a combined tile with
+    # the last 128; 177 and 200 leave a separate transposed tile, 100 and 20 a
+    # transposed tile alone, 128 a plain one.  FP8: per-row scales in the epilogue.
+    counts = np.array([129, 150, 176, 177, 128, 100, 304, 20, 200])
+    wl = synth.Workload("combo", T=int(counts.sum()), d=256, N=len(counts), k=1, H=384, act=act,
+                        dtype="bf16", gate_mode="R", dispatch="fp8" if fp8 else "", seed=29)
+    assert wl.T < 512 * wl.N
+    dev, host = upload_inputs(wl)
+    cfg = cfg_of(wl)
+    ws = moe.workspace(cfg)
+    offsets = np.concatenate([[0], np.cumsum(counts)]).astype(np.int32)
+    if fp8:
+        q, sc = oracle.quantize_rows(host["x"])
+        xp = torch.from_numpy(q).cuda()
+        xs = torch.from_numpy(sc).cuda()
+        xin = oracle.dequantize_rows(q, sc)
+    else:
+        xp, xs = dev["x"], None
+        xin = oracle.decode(host["x"])
+    yp = torch.zeros((wl.T, wl.d), dtype=torch.bfloat16, device="cuda")
+    moe.moe_expert_ffn(cfg, xp, xs, torch.from_numpy(offsets).cuda(), dev["W1"], dev.get("W3"),
+                       dev["W2"], yp, ws)
+    assert moe.moe_check_status(ws)[0] == moe.MOE_OK
+    got = to_f64(yp)
+    exp_of_row = np.repeat(np.arange(wl.N), counts)
+    want = np.empty((wl.T, wl.d))
+    for r in range(wl.T):
+        e = exp_of_row[r]
+        want[r] = oracle.ffn_row(xin[r], host["W1"][e], host["W3"][e] if act == "swiglu" else None,
+                                 host["W2"][e], act)
+    tol = 5e-3   # the oracle takes the same dequantised rows, so FP8 adds no error here
+    for e in range(wl.N):
+        lo, hi = offsets[e], offsets[e + 1]
+        assert rel_l2(got[lo:hi], want[lo:hi]) <= tol, (e, "all rows")
+        tail = lo + (counts[e] // 128) * 128
+        if hi > tail and counts[e] > 128:
+            assert rel_l2(got[tail:hi], want[tail:hi]) <= tol, (e, "rows past the last 128")

@@ -26,6 +26,13 @@
 //     accumulators, so the epilogue of one tile overlaps the MMAs of the next;
 //   - tile order inside a group: m fastest, so CTAs running at the same time
 //     share the weight tile through L2;
+//   - a group that ends a few rows past a multiple of 128 (at most
+//     kComboMaxRows) has those rows computed in the same tile as its last
+//     128 rows ("combined" tile): one stage carries the weight block, the 128
+//     rows and the leftover rows; one MMA covers the 128 rows, a transposed
+//     MMA (weights as M, leftover rows as N) the rest, into the second TMEM
+//     accumulator.  The weight block is then streamed once for both, where a
+//     separate short tile would run at its own pace and read it again;
 //   - every mbarrier wait is bounded in time; on expiry the kernel records a
 //     status bit, tells the other roles to stop, waits (bounded) for its own
 //     copies and MMAs in flight, frees TMEM and returns.
@@ -58,16 +65,24 @@ struct GemmParams {
     uint32_t *status;
 };
 
+// Leftover rows a combined tile takes (multiple of 16; 256-column tiles only).
+constexpr int kComboMaxRows = 48;
+
 template <int BN, int EPI>
 struct Geometry {
     static constexpr int OUTN = (EPI == EPI_SWIGLU) ? BN / 2 : BN;
     static constexpr int B_STAGE_BYTES = BN * BK * 2;
-    static constexpr int STAGE_BYTES = A_STAGE_BYTES + B_STAGE_BYTES;
+    static constexpr int AB_BYTES = A_STAGE_BYTES + B_STAGE_BYTES;
+    static constexpr int REM_ROWS = (BN >= 256) ? kComboMaxRows : 0;   // combined tiles
+    static constexpr int REM_BYTES = REM_ROWS * BK * 2;
+    static constexpr int STAGE_BYTES = AB_BYTES + REM_BYTES;
     static constexpr int STAGES = (BN >= 256) ? 4 : ((BN >= 128) ? 6 : 8);
     static constexpr int TMEM_COLS = (2 * BN <= 32) ? 32 : (2 * BN <= 64 ? 64 : (2 * BN <= 128 ? 128 : (2 * BN <= 256 ? 256 : 512)));
     // shared memory: [1 KB align slack][stages][barriers + tables]
     static constexpr int AUX_BYTES = 8 * (2 * STAGES + 5) + 16 + 8 * (kMaxGroups + 2);
     static constexpr int SMEM_BYTES = 1024 + STAGES * STAGE_BYTES + AUX_BYTES;
+    static_assert(SMEM_BYTES <= 232448, "shared memory per block");
+    static_assert(STAGE_BYTES % 1024 == 0, "stages keep the 1024-byte swizzle alignment");
 };
 
 // A partial tile of at most kSwapMaxRows rows runs "swapped": the weight rows
@@ -84,14 +99,29 @@ struct TileInfo {
     bool swap;
     int32_t ntok;   // swapped tiles: MMA N (rows_valid rounded up to 16)
     int32_t ks, kb0, kb1;   // K split index and its k-block range
+    bool combo;             // combined tile: rows_valid = 128 plus rem_rows more
+    int32_t rem_rows, rem_ntok;
 };
+
+// m tiles of a group of `rows` rows when up to rem_max leftover rows ride
+// in the last full tile (rem_max = 0: one tile per 128 rows or part of it).
+__host__ __device__ __forceinline__ int m_tiles_of(int rows, int rem_max)
+{
+    if (rows <= 0)
+        return 0;
+    if (rows <= BM)
+        return 1;
+    const int q = rows / BM;
+    const int rem = rows - q * BM;
+    return (rem == 0 || rem <= rem_max) ? q : q + 1;
+}
 
 // Locate tile t: prefix[g] <= t < prefix[g+1].  Inside a group the order is
 // (K split, n tile, m tile) with m fastest, so CTAs running side by side share
 // the weight tile through L2.
 __device__ __forceinline__ TileInfo tile_info(int t, const int32_t *s_prefix,
                                               const int32_t *s_off, int G, int n_tiles,
-                                              int outn, int ksplit, int KB)
+                                              int outn, int ksplit, int KB, int rem_max)
 {
     int lo = 0, hi = G;  // find largest g with prefix[g] <= t
     while (hi - lo > 1) {
@@ -103,7 +133,7 @@ __device__ __forceinline__ TileInfo tile_info(int t, const int32_t *s_prefix,
     }
     int g = lo;
     int rows_g = s_off[g + 1] - s_off[g];
-    int mt_g = (rows_g + BM - 1) / BM;
+    int mt_g = m_tiles_of(rows_g, rem_max);
     int local = t - s_prefix[g];
     const int per_split = mt_g * n_tiles;
     const int ks = local / per_split;
@@ -115,7 +145,11 @@ __device__ __forceinline__ TileInfo tile_info(int t, const int32_t *s_prefix,
     ti.row0 = s_off[g] + m_tile * BM;
     ti.rows_valid = min(BM, rows_g - m_tile * BM);
     ti.n0 = n_tile * outn;
-    ti.swap = ti.rows_valid <= kSwapMaxRows;
+    const int rest = rows_g - (m_tile + 1) * BM;   // rows past this tile (last tile: <= rem_max)
+    ti.combo = (m_tile == mt_g - 1) && rest > 0;
+    ti.rem_rows = ti.combo ? rest : 0;
+    ti.rem_ntok = (ti.rem_rows + 15) & ~15;
+    ti.swap = !ti.combo && ti.rows_valid <= kSwapMaxRows;
     ti.ntok = (ti.rows_valid + 15) & ~15;
     ti.ks = ks;
     ti.kb0 = static_cast<int>((static_cast<int64_t>(ks) * KB) / ksplit);
@@ -242,7 +276,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             if (g < G) {
                 int rows = s_off[g + 1] - s_off[g];
                 rows = rows > 0 ? rows : 0;
-                sum += ((rows + BM - 1) / BM) * n_tiles * p.ksplit;
+                sum += m_tiles_of(rows, Geo::REM_ROWS) * n_tiles * p.ksplit;
             }
         }
         int incl = sum;
@@ -259,7 +293,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                 if (g < G) {
                     int rows = s_off[g + 1] - s_off[g];
                     rows = rows > 0 ? rows : 0;
-                    run += ((rows + BM - 1) / BM) * n_tiles * p.ksplit;
+                    run += m_tiles_of(rows, Geo::REM_ROWS) * n_tiles * p.ksplit;
                 }
             }
         }
@@ -282,7 +316,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             // this CTA's own (tile, k-block) sequence, weights only
             int pf_t = blockIdx.x, pf_kb = 0, pf_kb1 = 0, pf_brow = 0;
             if (pf_t < total_tiles) {
-                const TileInfo pi = tile_info(pf_t, s_prefix, s_off, G, n_tiles, OUTN, p.ksplit, KB);
+                const TileInfo pi = tile_info(pf_t, s_prefix, s_off, G, n_tiles, OUTN, p.ksplit, KB, Geo::REM_ROWS);
                 pf_brow = pi.g * p.n_out + pi.n0;
                 pf_kb = pi.kb0;
                 pf_kb1 = pi.kb1;
@@ -296,7 +330,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                 if (++pf_kb >= pf_kb1) {
                     pf_t += gridDim.x;
                     if (pf_t < total_tiles) {
-                        const TileInfo pi = tile_info(pf_t, s_prefix, s_off, G, n_tiles, OUTN, p.ksplit, KB);
+                        const TileInfo pi = tile_info(pf_t, s_prefix, s_off, G, n_tiles, OUTN, p.ksplit, KB, Geo::REM_ROWS);
                         pf_brow = pi.g * p.n_out + pi.n0;
                         pf_kb = pi.kb0;
                         pf_kb1 = pi.kb1;
@@ -306,11 +340,13 @@ __global__ void __launch_bounds__(kThreads, 1)
             for (int i = 0; i < kPrefetchAhead; ++i)
                 prefetch_next();
             for (int t = blockIdx.x; t < total_tiles && ok; t += gridDim.x) {
-                const TileInfo ti = tile_info(t, s_prefix, s_off, G, n_tiles, OUTN, p.ksplit, KB);
+                const TileInfo ti = tile_info(t, s_prefix, s_off, G, n_tiles, OUTN, p.ksplit, KB, Geo::REM_ROWS);
                 const int brow = ti.g * p.n_out + ti.n0;
                 const int a_boxes = ti.ntok / 16;          // swapped tile: 16-row boxes
-                const uint32_t bytes = ti.swap ? (a_boxes * 16 * BK * 2 + Geo::B_STAGE_BYTES)
-                                               : Geo::STAGE_BYTES;
+                const int r_boxes = ti.rem_ntok / 16;      // combined tile: leftover rows
+                const uint32_t bytes =
+                    ti.swap ? (a_boxes * 16 * BK * 2 + Geo::B_STAGE_BYTES)
+                            : (Geo::AB_BYTES + r_boxes * 16 * BK * 2);
                 for (int kb = ti.kb0; kb < ti.kb1; ++kb) {
                     if (!mbar_wait_bounded(&empty[s], ph ^ 1u, s_abort)) {
                         set_status(p.status, DEV_TIMEOUT_PRODUCER);
@@ -327,6 +363,9 @@ __global__ void __launch_bounds__(kThreads, 1)
                                         ti.row0 + 16 * b);
                     } else {
                         tma_load_2d(sa, &tmA, &full[s], kb * BK, ti.row0);
+                        for (int b = 0; b < r_boxes; ++b)   // leftover rows after the B block
+                            tma_load_2d(sb + Geo::B_STAGE_BYTES + b * 16 * BK * 2, &tmA16,
+                                        &full[s], kb * BK, ti.row0 + BM + 16 * b);
                     }
                     if (EPI == EPI_SWIGLU) {
                         tma_load_2d(sb, &tmB, &full[s], kb * BK, brow);
@@ -360,18 +399,24 @@ __global__ void __launch_bounds__(kThreads, 1)
             uint32_t ph = 0;
             int it = 0;
             bool ok = true;
-            for (int t = blockIdx.x; t < total_tiles && ok; t += gridDim.x, ++it) {
-                const TileInfo ti = tile_info(t, s_prefix, s_off, G, n_tiles, OUTN, p.ksplit, KB);
+            for (int t = blockIdx.x; t < total_tiles && ok; t += gridDim.x) {
+                const TileInfo ti = tile_info(t, s_prefix, s_off, G, n_tiles, OUTN, p.ksplit, KB, Geo::REM_ROWS);
                 const uint32_t idesc_s = idesc_bf16_f32(128, ti.ntok);
+                const uint32_t idesc_r = idesc_bf16_f32(128, ti.rem_ntok > 0 ? ti.rem_ntok : 16);
+                // accumulator(s): a combined tile takes the next two
                 const int a = it & 1;
                 const uint32_t aph = (it >> 1) & 1;
-                if (!mbar_wait_bounded(&acc_empty[a], aph ^ 1u, s_abort)) {
+                const int a2 = (it + 1) & 1;
+                const uint32_t aph2 = ((it + 1) >> 1) & 1;
+                if (!mbar_wait_bounded(&acc_empty[a], aph ^ 1u, s_abort) ||
+                    (ti.combo && !mbar_wait_bounded(&acc_empty[a2], aph2 ^ 1u, s_abort))) {
                     set_status(p.status, DEV_TIMEOUT_MMA);
                     *s_abort = 1;
                     break;
                 }
                 tc_fence_after();
                 const uint32_t d_tmem = tmem_base + a * BN;
+                const uint32_t d_rem = tmem_base + a2 * BN;
                 for (int kb = ti.kb0; kb < ti.kb1; ++kb) {
                     if (!mbar_wait_bounded(&full[s], ph, s_abort)) {
                         set_status(p.status, DEV_TIMEOUT_MMA);
@@ -382,12 +427,24 @@ __global__ void __launch_bounds__(kThreads, 1)
                     tc_fence_after();
                     const uint32_t sa = smem_u32(stage_base + s * Geo::STAGE_BYTES);
                     const uint32_t sb = sa + A_STAGE_BYTES;
+                    const uint32_t sr = sb + Geo::B_STAGE_BYTES;
                     if (!ti.swap) {
 #pragma unroll
                         for (int kk = 0; kk < BK / 16; ++kk)
                             tc_mma_bf16(d_tmem, sdesc_kmajor_sw128(sa + kk * 32),
                                         sdesc_kmajor_sw128(sb + kk * 32), idesc_n,
                                         (kb > ti.kb0 || kk > 0) ? 1u : 0u);
+                        if (ti.combo) {
+                            // leftover rows, transposed, into the second accumulator
+#pragma unroll
+                            for (int kk = 0; kk < BK / 16; ++kk)
+#pragma unroll
+                                for (int h = 0; h < HALVES; ++h)
+                                    tc_mma_bf16(d_rem + h * 128,
+                                                sdesc_kmajor_sw128(sb + h * 128 * BK * 2 + kk * 32),
+                                                sdesc_kmajor_sw128(sr + kk * 32), idesc_r,
+                                                (kb > ti.kb0 || kk > 0) ? 1u : 0u);
+                        }
                     } else {
                         // D^T: weight rows are the MMA's M, the tile's tokens its N
 #pragma unroll
@@ -405,17 +462,21 @@ __global__ void __launch_bounds__(kThreads, 1)
                         ph ^= 1u;
                     }
                 }
-                if (ok)
+                if (ok) {
                     tc_commit(&acc_full[a]);
+                    if (ti.combo)
+                        tc_commit(&acc_full[a2]);
+                }
+                it += ti.combo ? 2 : 1;
             }
         }
     } else {
         // ================= epilogue (warps 2..5) =================
         const int q = warp & 3;                 // TMEM lane quarter of this warp
         const int r_in_tile = q * 32 + lane;
-        int it = 0;
-        for (int t = blockIdx.x; t < total_tiles; t += gridDim.x, ++it) {
-            const TileInfo ti = tile_info(t, s_prefix, s_off, G, n_tiles, OUTN, p.ksplit, KB);
+        // one accumulator's worth: a plain or transposed tile (or part of a
+        // combined one) from accumulator it & 1; false when its wait failed
+        auto part = [&](const TileInfo &ti, int it) -> bool {
             const int a = it & 1;
             const uint32_t aph = (it >> 1) & 1;
             const bool got = mbar_wait_bounded(&acc_full[a], aph, s_abort);
@@ -424,7 +485,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                     set_status(p.status, DEV_TIMEOUT_EPILOGUE);
                     *s_abort = 1;
                 }
-                break;
+                return false;
             }
             tc_fence_after();
             const uint32_t tacc = tmem_base + (static_cast<uint32_t>(q * 32) << 16) + a * BN;
@@ -507,6 +568,25 @@ __global__ void __launch_bounds__(kThreads, 1)
             }
             tc_fence_before();
             mbar_arrive(&acc_empty[a]);
+            return true;
+        };
+        int it = 0;
+        for (int t = blockIdx.x; t < total_tiles; t += gridDim.x) {
+            const TileInfo ti = tile_info(t, s_prefix, s_off, G, n_tiles, OUTN, p.ksplit, KB, Geo::REM_ROWS);
+            if (!part(ti, it))
+                break;
+            if (ti.combo) {
+                // the leftover rows of a combined tile, transposed, in the next accumulator
+                TileInfo tr = ti;
+                tr.row0 = ti.row0 + BM;
+                tr.rows_valid = ti.rem_rows;
+                tr.ntok = ti.rem_ntok;
+                tr.swap = true;
+                tr.combo = false;
+                if (!part(tr, it + 1))
+                    break;
+            }
+            it += ti.combo ? 2 : 1;
         }
     }
 
