@@ -54,7 +54,7 @@ def _load():
         build()
         lib = ctypes.CDLL(_SO)
         lib.orc_router_logits.argtypes = [_i64, _i64, _i32, _i32, _p, _i32, _p, _i32, _p, _p]
-        lib.orc_topk_gate.argtypes = [_i64, _i32, _i32, _i32, _i32, _p, _p, _p, _p]
+        lib.orc_topk_gate.argtypes = [_i64, _i32, _i32, _i32, _i32, _p, _p, _p, _p, _i32, _i32]
         lib.orc_dispatch.argtypes = [_i64, _i32, _i32, _f64, _p, _p, _p, _p, _p, _p, _p]
         lib.orc_dispatch.restype = _i64
         lib.orc_aux.argtypes = [_i64, _i32, _i32, _f64, _p, _p, _p, _p, _p]
@@ -110,15 +110,25 @@ def router_logits(x: np.ndarray, Wg: np.ndarray, bias: np.ndarray | None = None,
     return out
 
 
-def topk_gate(logits: np.ndarray, k: int, gate_mode: str, renormalize: bool = False):
-    """(idx [T,k] int32, gate [T,k] fp64, probs [T,N] fp64) from fp64 logits."""
+def topk_gate(logits: np.ndarray, k: int, gate_mode: str, renormalize: bool = False,
+              n_groups: int = 0, topk_groups: int = 0):
+    """(idx [T,k] int32, gate [T,k] fp64, probs [T,N] fp64) from fp64 logits.
+
+    n_groups > 1 and topk_groups < n_groups: node-limited routing ("MoE: what it
+    costs to train and serve", Limit how many machines a token touches) -- the
+    top-k is taken among the experts of the topk_groups nodes (blocks of
+    N / n_groups consecutive experts) with the largest sums of their
+    ceil(k / topk_groups) highest router probabilities."""
     logits = _c(logits.astype(np.float64))
     T, N = logits.shape
     idx = np.empty((T, k), dtype=np.int32)
     gate = np.empty((T, k), dtype=np.float64)
     probs = np.empty((T, N), dtype=np.float64)
+    if n_groups > 1 and topk_groups < n_groups:
+        assert N % n_groups == 0 and 1 <= topk_groups and k <= topk_groups * (N // n_groups)
     _load().orc_topk_gate(T, N, k, GATE_R if gate_mode == "R" else GATE_F, int(renormalize),
-                          logits.ctypes.data, idx.ctypes.data, gate.ctypes.data, probs.ctypes.data)
+                          logits.ctypes.data, idx.ctypes.data, gate.ctypes.data, probs.ctypes.data,
+                          int(n_groups), int(topk_groups))
     return idx, gate, probs
 
 
@@ -247,7 +257,8 @@ def layer_rows(act: str, xin: np.ndarray, idx: np.ndarray, gate: np.ndarray, dro
 def route(wl, x: np.ndarray, Wg: np.ndarray, bias=None) -> dict:
     """Router + top-k + aux + dispatch for every token of workload ``wl``."""
     logits = router_logits(x, Wg, bias)
-    idx, gate, probs = topk_gate(logits, wl.k, wl.gate_mode, wl.renormalize)
+    idx, gate, probs = topk_gate(logits, wl.k, wl.gate_mode, wl.renormalize,
+                                 wl.n_groups, wl.topk_groups)
     disp = dispatch(idx, wl.N, wl.capacity_factor)
     f, pm, laux = aux(disp["counts"], probs, wl.k, wl.aux_alpha)
     out = dict(logits=logits, idx=idx, gate=gate, probs=probs, f=f, p_mean=pm, L_aux=laux)

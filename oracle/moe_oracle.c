@@ -85,14 +85,34 @@ void orc_router_logits(int64_t t0, int64_t t1, int d, int N,
 /*   they are divided by their sum.                                    */
 /* probs (optional, [nt][N]) always receives the full softmax over N   */
 /* (the router probability used by the aux loss, [P5] Load balancing).*/
+/*                                                                     */
+/* Node-limited routing ([P4] "Limit how many machines a token         */
+/* touches": each token may go to at most a few nodes, chosen by the   */
+/* sum of the highest expert scores on each node).  READING: the N     */
+/* experts sit on n_groups nodes of N / n_groups consecutive experts;  */
+/* an expert's score is its router probability softmax(l)_e; a node's  */
+/* score is the sum of its m = ceil(k / topk_groups) highest; nodes are */
+/* ranked by score, largest first, the lower node index first on equal */
+/* scores; the top-k is then taken, in the order above, among the      */
+/* experts of the first topk_groups nodes only.  n_groups <= 1 or       */
+/* topk_groups >= n_groups: no limit.                                  */
 /* ------------------------------------------------------------------ */
 void orc_topk_gate(int64_t nt, int N, int k, int gate_mode, int renormalize,
-                   const double *logits, int32_t *idx, double *gate, double *probs)
+                   const double *logits, int32_t *idx, double *gate, double *probs,
+                   int n_groups, int topk_groups)
 {
+    const int limited = n_groups > 1 && topk_groups < n_groups;
+    const int gsize = limited ? N / n_groups : N;
+    const int m = limited ? (k + topk_groups - 1) / topk_groups : 0;
     #pragma omp parallel
     {
         int *ord = (int *)malloc(sizeof(int) * (size_t)N);
+        int *sel = (int *)malloc(sizeof(int) * (size_t)N);
         double *p = (double *)malloc(sizeof(double) * (size_t)N);
+        double *gscore = (double *)malloc(sizeof(double) * (size_t)(n_groups > 0 ? n_groups : 1));
+        int *gcnt = (int *)malloc(sizeof(int) * (size_t)(n_groups > 0 ? n_groups : 1));
+        int *gord = (int *)malloc(sizeof(int) * (size_t)(n_groups > 0 ? n_groups : 1));
+        char *allowed = (char *)malloc((size_t)(n_groups > 0 ? n_groups : 1));
         #pragma omp for schedule(static)
         for (int64_t t = 0; t < nt; ++t) {
             const double *l = logits + t * (int64_t)N;
@@ -116,24 +136,63 @@ void orc_topk_gate(int64_t nt, int N, int k, int gate_mode, int renormalize,
             if (probs)
                 memcpy(probs + t * (int64_t)N, p, sizeof(double) * (size_t)N);
 
+            /* the experts the token may use, in the order above */
+            int nsel = 0;
+            if (!limited) {
+                for (int e = 0; e < N; ++e)
+                    sel[nsel++] = ord[e];
+            } else {
+                for (int g = 0; g < n_groups; ++g) {
+                    gscore[g] = 0.0;
+                    gcnt[g] = 0;
+                }
+                for (int r = 0; r < N; ++r) {       /* each node's m highest, largest first */
+                    const int e = ord[r], g = e / gsize;
+                    if (gcnt[g] < m) {
+                        gscore[g] += p[e];
+                        ++gcnt[g];
+                    }
+                }
+                for (int g = 0; g < n_groups; ++g) { /* stable insertion sort of the nodes */
+                    int pos = g;
+                    while (pos > 0 && gscore[gord[pos - 1]] < gscore[g]) {
+                        gord[pos] = gord[pos - 1];
+                        --pos;
+                    }
+                    gord[pos] = g;
+                }
+                for (int g = 0; g < n_groups; ++g)
+                    allowed[g] = 0;
+                for (int j = 0; j < topk_groups; ++j)
+                    allowed[gord[j]] = 1;
+                for (int r = 0; r < N; ++r)
+                    if (allowed[ord[r] / gsize])
+                        sel[nsel++] = ord[r];
+            }
+
             for (int j = 0; j < k; ++j)
-                idx[t * k + j] = ord[j];
+                idx[t * k + j] = sel[j];
             if (gate_mode == ORC_GATE_R) {
-                double top = l[ord[0]], s = 0.0;
+                double top = l[sel[0]], s = 0.0;
                 for (int j = 0; j < k; ++j)
-                    s += exp(l[ord[j]] - top);
+                    s += exp(l[sel[j]] - top);
                 for (int j = 0; j < k; ++j)
-                    gate[t * k + j] = exp(l[ord[j]] - top) / s;
+                    gate[t * k + j] = exp(l[sel[j]] - top) / s;
             } else {
                 double s = 0.0;
                 for (int j = 0; j < k; ++j)
-                    s += p[ord[j]];
+                    s += p[sel[j]];
                 for (int j = 0; j < k; ++j)
-                    gate[t * k + j] = renormalize ? p[ord[j]] / s : p[ord[j]];
+                    gate[t * k + j] = renormalize ? p[sel[j]] / s : p[sel[j]];
             }
         }
         free(ord);
+        free(sel);
         free(p);
+        free(gscore);
+        free(gcnt);
+        free(gord);
+        free(allowed);
     }
 }
 

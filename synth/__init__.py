@@ -105,6 +105,8 @@ class Workload:
     aux_alpha: float = 0.01
     bias_std: float = 0.0   # > 0: per-expert logit bias ~ N(0, bias_std^2)
     seed: int = 0
+    n_groups: int = 0       # > 1: experts on n_groups nodes of N / n_groups consecutive experts
+    topk_groups: int = 0    # ... and a token may use at most topk_groups of them
 
     @property
     def dispatch_dtype(self) -> str:
@@ -134,7 +136,15 @@ DEEPSEEK = Workload("deepseek-v3-shaped T4096 d7168 N256+1 k8 H2048 swiglu bf16 
 GROK = Workload("grok1-shaped decode T32 d6144 N8 k2 H32768 swiglu bf16", T=32, d=6144, N=8, k=2,
                 H=32768, act="swiglu", dtype="bf16", gate_mode="R", seed=4)
 
-WORKLOADS = {"tiny": TINY_F32, "mixtral": MIXTRAL, "switch": SWITCH, "deepseek": DEEPSEEK, "grok": GROK}
+# The DeepSeek-shaped layer with node-limited routing: 8 nodes of 32 experts,
+# at most 4 nodes per token ("MoE: what it costs to train and serve", Limit how
+# many machines a token touches).
+DEEPSEEK_NODE_LIMITED = DEEPSEEK.with_(
+    name="deepseek-v3-shaped node-limited (8 nodes x 32 experts, <= 4 nodes per token)",
+    n_groups=8, topk_groups=4)
+
+WORKLOADS = {"tiny": TINY_F32, "mixtral": MIXTRAL, "switch": SWITCH, "deepseek": DEEPSEEK, "grok": GROK,
+             "deepseek-nl": DEEPSEEK_NODE_LIMITED}
 
 
 def tensor_specs(wl: Workload):

@@ -100,3 +100,69 @@ def test_switch_style_top1_weight_is_pmax_not_one():
     assert abs(gate[0, 0] - p[2] / p.sum()) < 1e-15
     _, gate_r, _ = oracle.topk_gate(logits, 1, "R")
     assert gate_r[0, 0] == 1.0
+
+
+# ---------------------------------------------------------------- node-limited routing
+def _golden(name):
+    vals = {}
+    with open(__file__.rsplit("/", 1)[0] + "/golden/" + name) as f:
+        for line in f:
+            if line.startswith("#") or ":" not in line:
+                continue
+            key, v = line.split(":", 1)
+            vals[key.strip()] = [float(a) for a in v.split()]
+    return vals
+
+
+def test_node_limited_worked_example():
+    g = _golden("node_limited_example.txt")
+    logits = np.array([g["logits"]])
+    k, ng, tg = int(g["k"][0]), int(g["n_groups"][0]), int(g["topk_groups"][0])
+    idx, gate, _ = oracle.topk_gate(logits, k, "F", renormalize=True, n_groups=ng, topk_groups=tg)
+    assert idx[0].tolist() == [int(v) for v in g["expect_idx"]]
+    plain, _, _ = oracle.topk_gate(logits, k, "F", renormalize=True)
+    assert plain[0].tolist() == [int(v) for v in g["plain_idx"]]
+    # renormalised gates are the softmax of the selected logits (library routine)
+    np.testing.assert_allclose(gate[0], scipy.special.softmax(logits[0, idx[0]]), rtol=1e-14)
+    # mode R picks the same experts with the same weights
+    idx_r, gate_r, _ = oracle.topk_gate(logits, k, "R", n_groups=ng, topk_groups=tg)
+    assert np.array_equal(idx_r, idx)
+    np.testing.assert_allclose(gate_r, gate, rtol=1e-14)
+
+
+@pytest.mark.parametrize("mode,renorm", [("R", False), ("F", False), ("F", True)])
+def test_node_limited_reduces_to_plain_topk(mode, renorm):
+    T, N, k = 200, 32, 4
+    logits = _rand(31, (T, N), 2.0).astype(np.float64)
+    logits[:, 7] = logits[:, 3]                      # exact ties across nodes
+    ref = oracle.topk_gate(logits, k, mode, renorm)
+    for ng, tg in [(1, 1), (4, 4), (8, 8), (N, k), (N, N)]:
+        # one node, every node allowed, or one expert per node with M >= k
+        got = oracle.topk_gate(logits, k, mode, renorm, n_groups=ng, topk_groups=tg)
+        for a, b in zip(got, ref):
+            assert np.array_equal(a, b), (ng, tg)
+
+
+def test_node_limited_deepseek_shape_invariants():
+    # 256 experts on 8 nodes of 32, top-8 from at most 4 nodes (the DeepSeek-V3
+    # setting the page describes)
+    T, N, k, ng, tg = 300, 256, 8, 8, 4
+    logits = _rand(32, (T, N), 1.0).astype(np.float64)
+    idx, gate, probs = oracle.topk_gate(logits, k, "F", True, n_groups=ng, topk_groups=tg)
+    plain, _, probs0 = oracle.topk_gate(logits, k, "F", True)
+    assert np.array_equal(probs, probs0)             # aux probabilities over all N, unchanged
+    nodes = idx // (N // ng)
+    assert all(len(set(r)) <= tg for r in nodes.tolist())
+    np.testing.assert_allclose(gate.sum(1), 1.0, rtol=1e-14)
+    # slot order: descending logit, distinct experts
+    sel = np.take_along_axis(logits, idx, 1)
+    assert np.all(np.diff(sel, axis=1) <= 0)
+    assert all(len(set(r)) == k for r in idx.tolist())
+    # the chosen experts are the k best of the chosen nodes (library sort)
+    for t in range(T):
+        allowed = np.isin(np.arange(N) // (N // ng), np.unique(nodes[t]))
+        cand = np.where(allowed)[0]
+        best = cand[np.lexsort((cand, -logits[t, cand]))][:k]
+        assert idx[t].tolist() == best.tolist()
+    # the limit binds for a good share of tokens
+    assert np.mean([len(set(r)) > tg for r in (plain // (N // ng)).tolist()]) > 0.2
