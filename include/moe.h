@@ -98,6 +98,20 @@ typedef struct moe_config {
     int32_t dtype;           /* MOE_F32 or MOE_BF16 for x, weights, y */
     int32_t dispatch_dtype;  /* == dtype, or MOE_FP8_E4M3 (bf16 layers only) */
     float   aux_alpha;       /* alpha of L_aux = alpha * N * sum_i f_i p_i */
+    /* Node-limited routing ("MoE: what it costs to train and serve", Limit how
+     * many machines a token touches: a token may go to at most a few nodes,
+     * chosen by the sum of the highest expert scores on each node).  With
+     * n_groups > 1 and topk_groups < n_groups the N experts sit on n_groups
+     * nodes of N / n_groups consecutive experts; a token uses at most
+     * topk_groups of them, those with the largest sums of their
+     * ceil(k / topk_groups) highest router probabilities (equal sums: lower
+     * node first), and its top-k is taken among those nodes' experts.
+     * Requires N % n_groups == 0, n_groups <= 32, 1 <= topk_groups,
+     * k <= topk_groups * N / n_groups, and gate mode R or renormalised mode F
+     * (plain mode F with nodes: MOE_ERR_UNSUPPORTED).  The aux statistics
+     * still use the softmax over all N.  0 / 0: no nodes. */
+    int32_t n_groups;
+    int32_t topk_groups;
 } moe_config;
 
 /* Bytes of workspace every entry point below needs for `cfg` (0 on an invalid

@@ -17,7 +17,8 @@ def cfg_of(wl: synth.Workload) -> moe.moe_config:
     return moe.make_config(wl.T, wl.d, wl.N, wl.k, wl.H, H_shared=wl.H_shared,
                            capacity_factor=wl.capacity_factor, gate_mode=wl.gate_mode,
                            renormalize=wl.renormalize, act=wl.act, dtype=wl.dtype,
-                           dispatch_dtype=wl.dispatch or None, aux_alpha=wl.aux_alpha)
+                           dispatch_dtype=wl.dispatch or None, aux_alpha=wl.aux_alpha,
+                           n_groups=wl.n_groups, topk_groups=wl.topk_groups)
 
 
 def tdtype(wl: synth.Workload):
@@ -103,6 +104,46 @@ def near_tie_tokens(logits: np.ndarray, idx: np.ndarray, k: int, rel: float = 1e
     srt = -np.sort(-logits, axis=1)
     a, b = srt[:, k - 1], srt[:, k]
     return np.abs(a - b) <= rel * np.maximum(np.abs(a), np.abs(b))
+
+
+def node_near_ties(probs: np.ndarray, k: int, n_groups: int, topk_groups: int,
+                   rel: float = 1e-3) -> np.ndarray:
+    """Node-limited routing: tokens whose topk_groups-th and next node scores
+    (sum of a node's ceil(k / topk_groups) highest probabilities) are within rel."""
+    T, N = probs.shape
+    S = N // n_groups
+    m = -(-k // topk_groups)
+    top = -np.sort(-probs.reshape(T, n_groups, S), axis=2)[:, :, :m].sum(2)
+    srt = -np.sort(-top, axis=1)
+    a, b = srt[:, topk_groups - 1], srt[:, topk_groups]
+    return np.abs(a - b) <= rel * np.maximum(a, b)
+
+
+def chosen_node_near_ties(logits: np.ndarray, idx: np.ndarray, k: int, n_groups: int,
+                          rel: float = 1e-3) -> np.ndarray:
+    """Node-limited routing: near-ties between the k-th and next logits among the
+    experts of the nodes the oracle chose."""
+    T, N = logits.shape
+    S = N // n_groups
+    masked = np.full_like(logits, -np.inf)
+    for t in range(T):
+        for g in np.unique(idx[t] // S):
+            masked[t, g * S:(g + 1) * S] = logits[t, g * S:(g + 1) * S]
+    srt = -np.sort(-masked, axis=1)
+    a, b = srt[:, k - 1], srt[:, k]
+    fin = np.isfinite(b)
+    out = np.zeros(T, bool)
+    out[fin] = np.abs(a[fin] - b[fin]) <= rel * np.maximum(np.abs(a[fin]), np.abs(b[fin]))
+    return out
+
+
+def route_near_ties(wl: synth.Workload, ref: dict) -> np.ndarray:
+    """Tokens whose routing may legitimately differ from the oracle's."""
+    tie = near_tie_tokens(ref["logits"], ref["idx"], wl.k)
+    if wl.n_groups > 1 and wl.topk_groups < wl.n_groups:
+        tie |= node_near_ties(ref["probs"], wl.k, wl.n_groups, wl.topk_groups)
+        tie |= chosen_node_near_ties(ref["logits"], ref["idx"], wl.k, wl.n_groups)
+    return tie
 
 
 def rel_l2(a: np.ndarray, b: np.ndarray) -> float:

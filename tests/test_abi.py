@@ -94,3 +94,18 @@ def test_entry_points_reject_bad_arguments_before_launch(lib):
     badc = moe.make_config(16, 64, 8, 9, 128)
     r = lib.moe_layer_forward(ctypes.byref(badc), *([None] * 17), 0, None)
     assert r == moe.MOE_ERR_INVALID_ARG
+
+
+def test_node_limited_config_validation(lib):
+    # host-only: invalid node layouts make the configuration invalid (0 bytes)
+    ok = dict(T=64, d=128, N=64, k=4, H=128, dtype="bf16", gate_mode="R", n_groups=8, topk_groups=2)
+    assert moe.moe_workspace_bytes(moe.make_config(**ok)) > 0
+    assert moe.moe_workspace_bytes(moe.make_config(**{**ok, "n_groups": 0, "topk_groups": 0})) > 0
+    for bad in ({"n_groups": 7},                          # N not a multiple of the nodes
+                {"N": 128, "n_groups": 64},               # more than 32 nodes
+                {"k": 8, "topk_groups": 1, "n_groups": 16},   # 4 experts allowed, k = 8
+                {"n_groups": -1}, {"topk_groups": -2}):
+        assert moe.moe_workspace_bytes(moe.make_config(**{**ok, **bad})) == 0, bad
+    # the C struct and its ctypes mirror agree on the appended fields
+    import ctypes
+    assert ctypes.sizeof(moe.moe_config) == 64

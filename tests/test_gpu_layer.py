@@ -11,7 +11,7 @@ import torch
 import oracle
 import synth
 import top_routing_expert_warp_b200 as moe
-from gpu_util import LayerRun, near_tie_tokens, rel_l2, to_f64, upload_inputs, y_tol
+from gpu_util import route_near_ties, LayerRun, near_tie_tokens, rel_l2, to_f64, upload_inputs, y_tol
 from test_gpu_stages import SMALL
 
 pytestmark = pytest.mark.gpu
@@ -21,7 +21,7 @@ def _check_layer(wl, run, host, tokens, x=None, get_expert=None, shared=None):
     ref = oracle.route(wl, host["x"], host["Wg"], host.get("bias"))
     T, k = wl.T, wl.k
     gi = run.topk_idx.cpu().numpy()
-    tie = near_tie_tokens(ref["logits"], ref["idx"], k)
+    tie = route_near_ties(wl, ref)
     ok_route = np.all(gi == ref["idx"], axis=1)
     assert np.all(ok_route | tie), "routing differs on a token that is not a near-tie"
     # tokens whose routing or drop state could be affected by a near-tie flip
@@ -76,14 +76,14 @@ def test_layer_deterministic(name):
 
 FULL = {"tiny": (synth.TINY_F32, 256), "mixtral": (synth.MIXTRAL, 48),
         "switch": (synth.SWITCH, 512), "deepseek": (synth.DEEPSEEK, 12),
-        "grok": (synth.GROK, 32)}
+        "grok": (synth.GROK, 32), "deepseek-nl": (synth.DEEPSEEK_NODE_LIMITED, 12)}
 
 
 @pytest.mark.slow
 @pytest.mark.parametrize("name", list(FULL))
 def test_layer_full_size_sampled(name):
     wl, nsamp = FULL[name]
-    big = name == "deepseek"
+    big = name.startswith("deepseek")
     dev, host = upload_inputs(wl, keep_host=not big)
     run = LayerRun(wl, dev)
     run()

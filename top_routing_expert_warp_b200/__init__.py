@@ -38,7 +38,8 @@ class moe_config(ctypes.Structure):
                 ("capacity_factor", ctypes.c_float), ("gate_mode", ctypes.c_int32),
                 ("renormalize", ctypes.c_int32), ("act", ctypes.c_int32),
                 ("dtype", ctypes.c_int32), ("dispatch_dtype", ctypes.c_int32),
-                ("aux_alpha", ctypes.c_float)]
+                ("aux_alpha", ctypes.c_float), ("n_groups", ctypes.c_int32),
+                ("topk_groups", ctypes.c_int32)]
 
 
 class MoeError(RuntimeError):
@@ -132,14 +133,14 @@ def _check(status: int, where: str):
 
 def make_config(T, d, N, k, H, *, H_shared=0, capacity_factor=0.0, gate_mode="R",
                 renormalize=False, act="swiglu", dtype="bf16", dispatch_dtype=None,
-                aux_alpha=0.01) -> moe_config:
+                aux_alpha=0.01, n_groups=0, topk_groups=0) -> moe_config:
     dt = {"f32": MOE_F32, "bf16": MOE_BF16}[dtype]
     dd = dt if dispatch_dtype in (None, "", dtype) else {"fp8": MOE_FP8_E4M3}[dispatch_dtype]
     return moe_config(int(T), int(d), int(N), int(k), int(H), int(H_shared),
                       float(capacity_factor),
                       MOE_GATE_TOPK_THEN_SOFTMAX if gate_mode == "R" else MOE_GATE_SOFTMAX_THEN_TOPK,
                       int(bool(renormalize)), MOE_ACT_RELU if act == "relu" else MOE_ACT_SWIGLU,
-                      dt, dd, float(aux_alpha))
+                      dt, dd, float(aux_alpha), int(n_groups), int(topk_groups))
 
 
 def moe_workspace_bytes(cfg: moe_config) -> int:

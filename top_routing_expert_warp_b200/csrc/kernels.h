@@ -95,6 +95,7 @@ struct RouterLaunch {
     int64_t T;
     int32_t d, N, k;
     int32_t gate_mode, renormalize;
+    int32_t n_groups, topk_groups;   // node-limited routing (0 / 0: off), checked by the ABI
     const float *logits_in;  // large-N path: fp32 partial logits [ksplit][T][N] from the GEMM
     int32_t ksplit;          // number of partial logit slices
     float *logits_out;       // optional fp32 logits (small-N path)

@@ -65,6 +65,12 @@ struct Layout {
         inv_row, drop, x_scale, x_gemm, h, y_perm, hs, ys, total;
 };
 
+// Node-limited routing in effect: more than one node and fewer allowed.
+bool node_limited(const moe_config &c)
+{
+    return c.n_groups > 1 && c.topk_groups < c.n_groups;
+}
+
 bool config_ok(const moe_config *c)
 {
     if (!c)
@@ -88,6 +94,13 @@ bool config_ok(const moe_config *c)
         return false;
     if (c->T * c->k > 0x7FFFFFFFll)
         return false;
+    if (c->n_groups < 0 || c->topk_groups < 0)
+        return false;
+    if (node_limited(*c)) {
+        if (c->n_groups > 32 || c->N % c->n_groups != 0 || c->topk_groups < 1 ||
+            c->k > c->topk_groups * (c->N / c->n_groups))
+            return false;
+    }
     if (c->dtype == MOE_F32) {
         // fp32 layers: CUDA-core router (N <= 16) and a row-staged SIMT GEMM
         if (c->N > moe::kRouterSmallMaxN || c->d > 12288 || c->H > 12288 || c->H_shared > 12288)
@@ -161,6 +174,10 @@ moe_status run_router(const moe_config &c, const void *x, const void *Wg, const 
                       float *logits, int32_t *topk_idx, float *topk_w, float *p_mean,
                       const Ws &w, cudaStream_t s)
 {
+    // with nodes, plain mode F would weigh excluded experts' tensor-core logits in
+    // its softmax denominator without recomputing them
+    if (node_limited(c) && c.gate_mode == MOE_GATE_SOFTMAX_THEN_TOPK && !c.renormalize)
+        return MOE_ERR_UNSUPPORTED;
     if (c.T == 0) {
         if (p_mean)
             MOE_CUDA(cudaMemsetAsync(p_mean, 0, c.N * sizeof(float), s));
@@ -178,6 +195,8 @@ moe_status run_router(const moe_config &c, const void *x, const void *Wg, const 
     R.k = c.k;
     R.gate_mode = c.gate_mode;
     R.renormalize = c.renormalize;
+    R.n_groups = node_limited(c) ? c.n_groups : 0;
+    R.topk_groups = node_limited(c) ? c.topk_groups : 0;
     R.topk_idx = topk_idx;
     R.topk_w = topk_w;
     R.p_part = w.at<double>(w.L.p_part);

@@ -111,10 +111,64 @@ __device__ __forceinline__ void unpack_chunk(const uint4 a, float (&xf)[8])
 // *my_psum.
 template <int NMAX>
 __device__ __forceinline__ void small_select(const double (&acc)[NMAX], int64_t t, int N, int k,
-                                             int gate_mode, int renorm, int lane,
+                                             int gate_mode, int renorm, int n_groups,
+                                             int topk_groups, int lane,
                                              int32_t *__restrict__ topk_idx,
                                              float *__restrict__ topk_w, double *my_psum)
 {
+    // node-limited routing: lane g scores node g (sum of its m highest
+    // probabilities, as exp(l - max), largest first), then the topk_groups
+    // best nodes (lower node first on equal scores) are the allowed ones
+    uint32_t allowed = 0xffffffffu;
+    if (n_groups > 1) {
+        const int S = N / n_groups;
+        const int m = (k + topk_groups - 1) / topk_groups;
+        double gmx = acc[0];
+#pragma unroll
+        for (int e = 1; e < NMAX; ++e)
+            if (e < N && acc[e] > gmx)
+                gmx = acc[e];
+        double gs = -1.0;
+        if (lane < n_groups) {
+            gs = 0.0;
+            uint32_t tk = 0;
+#pragma unroll 1
+            for (int r = 0; r < m; ++r) {
+                int bi = -1;
+                double bv = 0.0;
+#pragma unroll
+                for (int e = 0; e < NMAX; ++e) {
+                    if (e < N && e / S == lane && !((tk >> e) & 1u) && (bi < 0 || acc[e] > bv)) {
+                        bi = e;
+                        bv = acc[e];
+                    }
+                }
+                tk |= 1u << bi;
+                gs += exp(bv - gmx);
+            }
+        }
+        uint32_t gtaken = 0;
+#pragma unroll 1
+        for (int j = 0; j < topk_groups; ++j) {
+            double v = (lane < n_groups && !((gtaken >> lane) & 1u)) ? gs : -1.0;
+            int gi = v >= 0.0 ? lane : 32;
+#pragma unroll
+            for (int o = 16; o > 0; o >>= 1) {
+                const double ov = __shfl_xor_sync(0xffffffffu, v, o);
+                const int oi = __shfl_xor_sync(0xffffffffu, gi, o);
+                if (ov > v || (ov == v && oi < gi)) {
+                    v = ov;
+                    gi = oi;
+                }
+            }
+            gtaken |= 1u << gi;
+        }
+        allowed = 0;
+#pragma unroll
+        for (int e = 0; e < NMAX; ++e)
+            if (e < N && ((gtaken >> (e / S)) & 1u))
+                allowed |= 1u << e;
+    }
     // top-k: strict comparison in ascending expert order -> lowest index wins
     uint32_t taken = 0;
     int sel[kMaxK];
@@ -128,7 +182,8 @@ __device__ __forceinline__ void small_select(const double (&acc)[NMAX], int64_t 
             double bv = 0.0;
 #pragma unroll
             for (int e = 0; e < NMAX; ++e) {
-                if (e < N && !((taken >> e) & 1u) && (bi < 0 || acc[e] > bv)) {
+                if (e < N && ((allowed >> e) & 1u) && !((taken >> e) & 1u) &&
+                    (bi < 0 || acc[e] > bv)) {
                     bi = e;
                     bv = acc[e];
                 }
@@ -180,9 +235,9 @@ template <bool BF16, int NMAX>
 __global__ void __launch_bounds__(kThreads)
     router_small_kernel(const void *__restrict__ xv, const void *__restrict__ wv,
                         const float *__restrict__ bias, int64_t T, int d, int N, int k,
-                        int gate_mode, int renorm, float *__restrict__ logits_out,
-                        int32_t *__restrict__ topk_idx, float *__restrict__ topk_w,
-                        double *__restrict__ p_part)
+                        int gate_mode, int renorm, int n_groups, int topk_groups,
+                        float *__restrict__ logits_out, int32_t *__restrict__ topk_idx,
+                        float *__restrict__ topk_w, double *__restrict__ p_part)
 {
     grid_dep_wait();
     __shared__ double s_p[kWarps][NMAX];
@@ -252,7 +307,8 @@ __global__ void __launch_bounds__(kThreads)
                     if (e < N && lane == e)
                         logits_out[t * N + e] = static_cast<float>(acc[e]);
             }
-            small_select<NMAX>(acc, t, N, k, gate_mode, renorm, lane, topk_idx, topk_w, &my_psum);
+            small_select<NMAX>(acc, t, N, k, gate_mode, renorm, n_groups, topk_groups, lane,
+                               topk_idx, topk_w, &my_psum);
         }
     }
     if (lane < NMAX)
@@ -272,6 +328,12 @@ __device__ __forceinline__ uint32_t order_key(float v)
 {
     const uint32_t u = __float_as_uint(v + 0.0f);
     return (u & 0x80000000u) ? ~u : (u | 0x80000000u);
+}
+
+// The float a key was made from.
+__device__ __forceinline__ float key_value(uint32_t key)
+{
+    return __uint_as_float((key & 0x80000000u) ? (key & 0x7fffffffu) : ~key);
 }
 
 // Compensated fp32 accumulator (hi + lo) of bf16 dot products; see DotAcc.
@@ -316,9 +378,9 @@ __global__ void __launch_bounds__(kThreads, NPL >= 8 ? 2 : 3)
     router_select_kernel(const float *__restrict__ part, int ksplit,
                          float *__restrict__ logits_out, const uint16_t *__restrict__ x,
                          const uint16_t *__restrict__ w, const float *__restrict__ bias, int64_t T,
-                         int d, int N, int k, int gate_mode, int renorm,
-                         int32_t *__restrict__ topk_idx, float *__restrict__ topk_w,
-                         double *__restrict__ p_part)
+                         int d, int N, int k, int gate_mode, int renorm, int n_groups,
+                         int topk_groups, int32_t *__restrict__ topk_idx,
+                         float *__restrict__ topk_w, double *__restrict__ p_part)
 {
     grid_dep_wait();
     extern __shared__ double s_pdyn[];  // [kWarps][N]
@@ -338,6 +400,13 @@ __global__ void __launch_bounds__(kThreads, NPL >= 8 ? 2 : 3)
 #pragma unroll
     for (int i = 0; i < NPL; ++i)
         psum[i] = 0.0f;
+    // node-limited routing: node of each of this lane's experts
+    int grp[NPL];
+    const int S = n_groups > 1 ? N / n_groups : N;
+#pragma unroll
+    for (int i = 0; i < NPL; ++i)
+        grp[i] = (lane + 32 * i) / S;
+    const int m_node = n_groups > 1 ? (k + topk_groups - 1) / topk_groups : 0;
 
     for (int64_t t = static_cast<int64_t>(blockIdx.x) * kWarps + warp; t < T;
          t += static_cast<int64_t>(gridDim.x) * kWarps) {
@@ -357,6 +426,61 @@ __global__ void __launch_bounds__(kThreads, NPL >= 8 ? 2 : 3)
                 lv[i] = v;
             }
         }
+        // node-limited routing: node g's score is the sum of its m_node
+        // highest probabilities (as exp(l - max), largest first), picked by
+        // warp reductions; lane g keeps it.  The topk_groups best nodes (lower
+        // node first on equal scores) hold the experts that may be chosen.
+        uint32_t allow = 0xffffffffu;   // bit i: expert lane + 32 i may be chosen
+        if (n_groups > 1) {
+            float lm = lv[0];
+#pragma unroll
+            for (int i = 1; i < NPL; ++i)
+                lm = fmaxf(lm, lv[i]);
+            const float gm = key_value(__reduce_max_sync(0xffffffffu, order_key(lm)));
+            float my_gs = -1.0f;
+#pragma unroll 1
+            for (int g = 0; g < n_groups; ++g) {
+                uint32_t tk = 0;
+                float sum = 0.0f;
+#pragma unroll 1
+                for (int r = 0; r < m_node; ++r) {
+                    float bv = -INFINITY;
+                    int be = -1;
+#pragma unroll
+                    for (int i = 0; i < NPL; ++i) {
+                        const int e = lane + 32 * i;
+                        if (e < N && grp[i] == g && !((tk >> i) & 1u) && (be < 0 || lv[i] > bv)) {
+                            bv = lv[i];
+                            be = e;
+                        }
+                    }
+                    const uint32_t key = be >= 0 ? order_key(bv) : 0u;
+                    const uint32_t top = __reduce_max_sync(0xffffffffu, key);
+                    const uint32_t eb = __reduce_min_sync(
+                        0xffffffffu, (be >= 0 && key == top) ? static_cast<uint32_t>(be) : 0xffffffffu);
+                    if (static_cast<int>(eb & 31u) == lane)
+                        tk |= 1u << (eb >> 5);
+                    sum += expf(key_value(top) - gm);
+                }
+                if (lane == g)
+                    my_gs = sum;
+            }
+            uint32_t gtaken = 0;
+#pragma unroll 1
+            for (int j = 0; j < topk_groups; ++j) {
+                const bool live = lane < n_groups && !((gtaken >> lane) & 1u);
+                const uint32_t key = live ? order_key(my_gs) : 0u;
+                const uint32_t top = __reduce_max_sync(0xffffffffu, key);
+                const uint32_t gi = __reduce_min_sync(
+                    0xffffffffu, (live && key == top) ? static_cast<uint32_t>(lane) : 0xffffffffu);
+                gtaken |= 1u << gi;
+            }
+            allow = 0;
+#pragma unroll
+            for (int i = 0; i < NPL; ++i)
+                if (lane + 32 * i < N && ((gtaken >> grp[i]) & 1u))
+                    allow |= 1u << i;
+        }
         // candidates: the KC best logits, best first.  Each round takes the
         // lane's best untaken logit (lowest index on a tie), then the warp's
         // largest (two warp reductions: the largest value, then the lowest
@@ -372,7 +496,8 @@ __global__ void __launch_bounds__(kThreads, NPL >= 8 ? 2 : 3)
 #pragma unroll
                 for (int i = 0; i < NPL; ++i) {
                     const int e = lane + 32 * i;
-                    if (e < N && !((taken >> i) & 1u) && (be < 0 || lv[i] > bv)) {
+                    if (e < N && ((allow >> i) & 1u) && !((taken >> i) & 1u) &&
+                        (be < 0 || lv[i] > bv)) {
                         bv = lv[i];
                         be = e;
                     }
@@ -565,21 +690,21 @@ cudaError_t launch_router_small(RouterLaunch &L, cudaStream_t stream)
     if (L.dtype == MOE_BF16) {
         if (L.N <= 8)
             launch_k(router_small_kernel<true, 8>, grid, kThreads, 0, stream, 
-                L.x, L.Wg, L.bias, L.T, L.d, L.N, L.k, L.gate_mode, L.renormalize,
-                L.logits_out, L.topk_idx, L.topk_w, L.p_part);
+                L.x, L.Wg, L.bias, L.T, L.d, L.N, L.k, L.gate_mode, L.renormalize, L.n_groups,
+                L.topk_groups, L.logits_out, L.topk_idx, L.topk_w, L.p_part);
         else
             launch_k(router_small_kernel<true, 16>, grid, kThreads, 0, stream, 
-                L.x, L.Wg, L.bias, L.T, L.d, L.N, L.k, L.gate_mode, L.renormalize,
-                L.logits_out, L.topk_idx, L.topk_w, L.p_part);
+                L.x, L.Wg, L.bias, L.T, L.d, L.N, L.k, L.gate_mode, L.renormalize, L.n_groups,
+                L.topk_groups, L.logits_out, L.topk_idx, L.topk_w, L.p_part);
     } else {
         if (L.N <= 8)
             launch_k(router_small_kernel<false, 8>, grid, kThreads, 0, stream, 
-                L.x, L.Wg, L.bias, L.T, L.d, L.N, L.k, L.gate_mode, L.renormalize,
-                L.logits_out, L.topk_idx, L.topk_w, L.p_part);
+                L.x, L.Wg, L.bias, L.T, L.d, L.N, L.k, L.gate_mode, L.renormalize, L.n_groups,
+                L.topk_groups, L.logits_out, L.topk_idx, L.topk_w, L.p_part);
         else
             launch_k(router_small_kernel<false, 16>, grid, kThreads, 0, stream, 
-                L.x, L.Wg, L.bias, L.T, L.d, L.N, L.k, L.gate_mode, L.renormalize,
-                L.logits_out, L.topk_idx, L.topk_w, L.p_part);
+                L.x, L.Wg, L.bias, L.T, L.d, L.N, L.k, L.gate_mode, L.renormalize, L.n_groups,
+                L.topk_groups, L.logits_out, L.topk_idx, L.topk_w, L.p_part);
     }
     count_launches(1);
     return cudaGetLastError();
@@ -591,7 +716,7 @@ void select_launch(RouterLaunch &L, int grid, size_t smem, cudaStream_t stream)
     launch_k(router_select_kernel<NPL, KCM>, grid, kThreads, smem, stream, 
         L.logits_in, L.ksplit, L.logits_out, static_cast<const uint16_t *>(L.x),
         static_cast<const uint16_t *>(L.Wg), L.bias, L.T, L.d, L.N, L.k, L.gate_mode,
-        L.renormalize, L.topk_idx, L.topk_w, L.p_part);
+        L.renormalize, L.n_groups, L.topk_groups, L.topk_idx, L.topk_w, L.p_part);
 }
 
 template <int NPL>
