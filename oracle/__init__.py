@@ -55,7 +55,7 @@ def _load():
         lib = ctypes.CDLL(_SO)
         lib.orc_router_logits.argtypes = [_i64, _i64, _i32, _i32, _p, _i32, _p, _i32, _p, _p]
         lib.orc_topk_gate.argtypes = [_i64, _i32, _i32, _i32, _i32, _p, _p, _p, _p, _i32, _i32]
-        lib.orc_dispatch.argtypes = [_i64, _i32, _i32, _f64, _p, _p, _p, _p, _p, _p, _p]
+        lib.orc_dispatch.argtypes = [_i64, _i32, _i32, _f64, _p, _p, _p, _p, _p, _p, _p, _i32, _i32, _p]
         lib.orc_dispatch.restype = _i64
         lib.orc_aux.argtypes = [_i64, _i32, _i32, _f64, _p, _p, _p, _p, _p]
         lib.orc_e4m3_decode.argtypes = [ctypes.c_uint8]
@@ -133,21 +133,29 @@ def topk_gate(logits: np.ndarray, k: int, gate_mode: str, renormalize: bool = Fa
 
 
 # ------------------------------------------------------------------- dispatch
-def dispatch(idx: np.ndarray, N: int, capacity_factor: float) -> dict:
-    """Local permutation: counts, kept, offsets, perm, inv_row, drop, R."""
+def dispatch(idx: np.ndarray, N: int, capacity_factor: float, fallback: bool = False,
+             slot_priority: bool = False) -> dict:
+    """Local permutation: counts, kept, offsets, perm, inv_row, drop, R, expert.
+
+    fallback: pairs over capacity go to a fallback expert N (offsets gets N + 2
+    entries) instead of being dropped; slot_priority: pairs are taken slot by
+    slot (every token's first choice first) instead of token by token
+    ("moe communication costs", Capacity factor and token dropping)."""
     idx = _c(idx.astype(np.int32))
     T, k = idx.shape
     counts = np.empty(N, np.int32)
     kept = np.empty(N, np.int32)
-    offsets = np.empty(N + 1, np.int32)
+    offsets = np.empty(N + 2 if fallback else N + 1, np.int32)
     perm = np.full(T * k, -1, np.int32)
     inv_row = np.empty(T * k, np.int32)
     drop = np.empty(T * k, np.uint8)
+    expert = np.empty(T * k, np.int32)
     R = _load().orc_dispatch(T, N, k, float(capacity_factor), idx.ctypes.data, counts.ctypes.data,
                              kept.ctypes.data, offsets.ctypes.data, perm.ctypes.data,
-                             inv_row.ctypes.data, drop.ctypes.data)
+                             inv_row.ctypes.data, drop.ctypes.data, int(bool(fallback)),
+                             int(bool(slot_priority)), expert.ctypes.data)
     return dict(counts=counts, kept=kept, offsets=offsets, perm=perm[:R], inv_row=inv_row,
-                drop=drop, R=int(R))
+                drop=drop, R=int(R), expert=expert)
 
 
 def aux(counts: np.ndarray, probs: np.ndarray, k: int, alpha: float):
@@ -259,7 +267,7 @@ def route(wl, x: np.ndarray, Wg: np.ndarray, bias=None) -> dict:
     logits = router_logits(x, Wg, bias)
     idx, gate, probs = topk_gate(logits, wl.k, wl.gate_mode, wl.renormalize,
                                  wl.n_groups, wl.topk_groups)
-    disp = dispatch(idx, wl.N, wl.capacity_factor)
+    disp = dispatch(idx, wl.N, wl.capacity_factor, wl.overflow == "fallback", wl.slot_priority)
     f, pm, laux = aux(disp["counts"], probs, wl.k, wl.aux_alpha)
     out = dict(logits=logits, idx=idx, gate=gate, probs=probs, f=f, p_mean=pm, L_aux=laux)
     out.update(disp)
@@ -274,13 +282,22 @@ def expert_inputs(wl, x_rows: np.ndarray):
     return decode(x_rows)
 
 
+def _effective_experts(wl, routing: dict) -> np.ndarray:
+    """[T, k] expert each pair runs on (the fallback N for re-routed pairs)."""
+    if "expert" not in routing:
+        return routing["idx"]
+    return np.where(routing["drop"].reshape(wl.T, wl.k) != 0, routing["idx"],
+                    routing["expert"].reshape(wl.T, wl.k)).astype(np.int32)
+
+
 def forward_rows(wl, inputs: dict, routing: dict, tokens) -> np.ndarray:
     """Layer output y [len(tokens), d] in fp64 for the listed tokens."""
     tokens = np.asarray(tokens, dtype=np.int64)
     x = inputs["x"]
     xr = x[tokens]
     xin = expert_inputs(wl, xr)
-    idx = routing["idx"][tokens]
+    # the expert each (token, slot) pair runs on: its own, or the fallback
+    idx = _effective_experts(wl, routing)[tokens]
     gate = routing["gate"][tokens]
     drop = routing["drop"].reshape(wl.T, wl.k)[tokens]
     W1, W2 = inputs["W1"], inputs["W2"]
@@ -300,7 +317,7 @@ def forward_rows_lazy(wl, x: np.ndarray, routing: dict, tokens, get_expert, shar
     tokens = np.asarray(tokens, dtype=np.int64)
     xr = x[tokens]
     xin = expert_inputs(wl, xr)
-    idx = routing["idx"][tokens]
+    idx = _effective_experts(wl, routing)[tokens]
     gate = routing["gate"][tokens]
     drop = routing["drop"].reshape(wl.T, wl.k)[tokens]
     used = sorted(set(int(e) for e, dr in zip(idx.ravel(), drop.ravel()) if not dr))

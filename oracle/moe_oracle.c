@@ -212,9 +212,23 @@ void orc_topk_gate(int64_t nt, int N, int k, int gate_mode, int renormalize,
 /* inv_row[t*k + j] = its row or -1; drop[t*k + j] = 1 if dropped.     */
 /* Returns R = offsets[N].                                             */
 /* ------------------------------------------------------------------ */
+/*                                                                     */
+/* The same paragraph: overflowing tokens are "either dropped ... or    */
+/* re-routed to a shared fallback expert".  READING (fallback != 0):    */
+/* the fallback is one more expert, index N, stored after the N routed */
+/* experts and without a capacity limit; every pair an expert cannot   */
+/* keep goes to it, in the order the pairs are taken, and keeps its    */
+/* gate weight.  offsets then has N + 2 entries (the fallback's rows   */
+/* are [offsets[N], offsets[N+1])).                                     */
+/* Order in which pairs are taken: token by token (t, then slot j),    */
+/* or, with slot_priority, slot by slot (every token's first choice    */
+/* before any token's second; READING of priority dropping for k > 1).  */
+/* expert_of[i]: the group pair i went to (its expert, N, or -1).       */
+/* ------------------------------------------------------------------ */
 int64_t orc_dispatch(int64_t T, int N, int k, double capacity_factor,
                      const int32_t *idx, int32_t *counts, int32_t *kept,
-                     int32_t *offsets, int32_t *perm, int32_t *inv_row, uint8_t *drop)
+                     int32_t *offsets, int32_t *perm, int32_t *inv_row, uint8_t *drop,
+                     int fallback, int slot_priority, int32_t *expert_of)
 {
     int64_t C = -1;
     if (capacity_factor > 0)
@@ -224,28 +238,39 @@ int64_t orc_dispatch(int64_t T, int N, int k, double capacity_factor,
     for (int64_t i = 0; i < T * k; ++i)
         counts[idx[i]] += 1;
     offsets[0] = 0;
+    int64_t over = 0;
     for (int e = 0; e < N; ++e) {
         kept[e] = (C < 0 || counts[e] <= C) ? counts[e] : (int32_t)C;
         offsets[e + 1] = offsets[e] + kept[e];
+        over += counts[e] - kept[e];
     }
+    if (fallback)
+        offsets[N + 1] = offsets[N] + (int32_t)over;
     int32_t *seen = (int32_t *)calloc((size_t)N, sizeof(int32_t));
-    for (int64_t t = 0; t < T; ++t) {          /* increasing token order */
-        for (int j = 0; j < k; ++j) {
-            int64_t i = t * k + j;
-            int e = idx[i];
-            int32_t r = seen[e]++;
-            if (C >= 0 && r >= C) {
-                drop[i] = 1;
-                inv_row[i] = -1;
-            } else {
-                drop[i] = 0;
-                inv_row[i] = offsets[e] + r;
-                perm[offsets[e] + r] = (int32_t)i;
-            }
+    int32_t fb = 0;
+    for (int64_t p = 0; p < T * k; ++p) {
+        const int64_t i = slot_priority ? (p % T) * k + p / T : p;
+        const int e = idx[i];
+        const int32_t r = seen[e]++;
+        if (C < 0 || r < C) {
+            drop[i] = 0;
+            inv_row[i] = offsets[e] + r;
+            perm[offsets[e] + r] = (int32_t)i;
+            expert_of[i] = e;
+        } else if (fallback) {
+            const int32_t row = offsets[N] + fb++;
+            drop[i] = 0;
+            inv_row[i] = row;
+            perm[row] = (int32_t)i;
+            expert_of[i] = N;
+        } else {
+            drop[i] = 1;
+            inv_row[i] = -1;
+            expert_of[i] = -1;
         }
     }
     free(seen);
-    return offsets[N];
+    return fallback ? offsets[N + 1] : offsets[N];
 }
 
 /* ------------------------------------------------------------------ */

@@ -107,6 +107,13 @@ class Workload:
     seed: int = 0
     n_groups: int = 0       # > 1: experts on n_groups nodes of N / n_groups consecutive experts
     topk_groups: int = 0    # ... and a token may use at most topk_groups of them
+    overflow: str = "drop"  # pairs over capacity: "drop", or "fallback" to expert N
+    slot_priority: bool = False   # capacity filled slot by slot (first choices first)
+
+    @property
+    def n_stored(self) -> int:
+        """Expert blocks in W1/W3/W2: the N routed experts (+ the fallback)."""
+        return self.N + (1 if self.overflow == "fallback" else 0)
 
     @property
     def dispatch_dtype(self) -> str:
@@ -143,8 +150,15 @@ DEEPSEEK_NODE_LIMITED = DEEPSEEK.with_(
     name="deepseek-v3-shaped node-limited (8 nodes x 32 experts, <= 4 nodes per token)",
     n_groups=8, topk_groups=4)
 
+# The Switch-shaped layer with its overflow re-routed to a fallback expert
+# instead of dropped ("moe communication costs", Capacity factor and token
+# dropping).
+SWITCH_FALLBACK = SWITCH.with_(
+    name="switch-shaped T8192 d1024 N128+fallback k1 H4096 relu bf16 cf1.25, overflow to a fallback expert",
+    overflow="fallback")
+
 WORKLOADS = {"tiny": TINY_F32, "mixtral": MIXTRAL, "switch": SWITCH, "deepseek": DEEPSEEK, "grok": GROK,
-             "deepseek-nl": DEEPSEEK_NODE_LIMITED}
+             "deepseek-nl": DEEPSEEK_NODE_LIMITED, "switch-fb": SWITCH_FALLBACK}
 
 
 def tensor_specs(wl: Workload):
@@ -153,10 +167,11 @@ def tensor_specs(wl: Workload):
              ("Wg", (wl.N, wl.d), 1.0 / math.sqrt(wl.d), wl.dtype)]
     if wl.bias_std > 0:
         specs.append(("bias", (wl.N,), wl.bias_std, "f32"))
-    specs.append(("W1", (wl.N, wl.H, wl.d), 1.0 / math.sqrt(wl.d), wl.dtype))
+    E = wl.n_stored
+    specs.append(("W1", (E, wl.H, wl.d), 1.0 / math.sqrt(wl.d), wl.dtype))
     if wl.act == "swiglu":
-        specs.append(("W3", (wl.N, wl.H, wl.d), 1.0 / math.sqrt(wl.d), wl.dtype))
-    specs.append(("W2", (wl.N, wl.d, wl.H), 1.0 / math.sqrt(wl.H), wl.dtype))
+        specs.append(("W3", (E, wl.H, wl.d), 1.0 / math.sqrt(wl.d), wl.dtype))
+    specs.append(("W2", (E, wl.d, wl.H), 1.0 / math.sqrt(wl.H), wl.dtype))
     if wl.H_shared > 0:
         specs.append(("Ws1", (wl.H_shared, wl.d), 1.0 / math.sqrt(wl.d), wl.dtype))
         if wl.act == "swiglu":

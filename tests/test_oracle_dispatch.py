@@ -1,8 +1,10 @@
 """Pins for the oracle's dispatch (counts, capacity, permutation) and aux statistics."""
 import math
+import os
 
 import numpy as np
 import pytest
+import scipy.special
 
 import oracle
 import synth
@@ -103,3 +105,108 @@ def test_laux_collapsed_router_is_alpha_times_n():
     f, pm, laux = oracle.aux(disp["counts"], probs, 1, 0.05)
     assert f[0] == 1.0
     assert abs(laux - 0.05 * N) < 1e-12
+
+
+# ------------------------------------------------- capacity variants (fallback expert, slot priority)
+def _golden(name):
+    vals = {}
+    with open(os.path.join(os.path.dirname(__file__), "golden", name)) as f:
+        for line in f:
+            if line.startswith("#") or ":" not in line:
+                continue
+            key, v = line.split(":", 1)
+            vals[key.strip()] = [float(a) for a in v.split()]
+    return vals
+
+
+def test_capacity_priority_worked_example():
+    g = _golden("capacity_priority_example.txt")
+    T, k, N = int(g["T"][0]), int(g["k"][0]), int(g["N"][0])
+    idx = np.array(g["idx"], np.int32).reshape(T, k)
+    cf = g["capacity_factor"][0]
+    ints = lambda key: [int(v) for v in g[key]]
+    tok = oracle.dispatch(idx, N, cf)
+    slot = oracle.dispatch(idx, N, cf, slot_priority=True)
+    assert tok["drop"].tolist() == ints("drop_token_order")
+    assert slot["drop"].tolist() == ints("drop_slot_order")
+    assert tok["perm"].tolist() == ints("perm_token_order")
+    assert slot["perm"].tolist() == ints("perm_slot_order")
+    for prio, key in [(False, "fallback_rows_token_order"), (True, "fallback_rows_slot_order")]:
+        fb = oracle.dispatch(idx, N, cf, fallback=True, slot_priority=prio)
+        assert fb["R"] == T * k and not fb["drop"].any()
+        assert fb["perm"][fb["offsets"][N]:fb["offsets"][N + 1]].tolist() == ints(key)
+        assert fb["expert"][ints(key)].tolist() == [N, N]
+
+
+def _brute(idx, N, C, slot_priority, fallback):
+    """Walk the pairs in the stated order with per-expert counters."""
+    T, k = idx.shape
+    order = [(t, j) for j in range(k) for t in range(T)] if slot_priority else \
+            [(t, j) for t in range(T) for j in range(k)]
+    seen = [0] * N
+    kept = {e: [] for e in range(N + 1)}
+    for t, j in order:
+        e = int(idx[t, j])
+        if C < 0 or seen[e] < C:
+            kept[e].append(t * k + j)
+        elif fallback:
+            kept[N].append(t * k + j)
+        seen[e] += 1
+    return [p for e in range(N + 1) for p in kept[e]]
+
+
+@pytest.mark.parametrize("slot_priority", [False, True])
+@pytest.mark.parametrize("fallback", [False, True])
+def test_capacity_variants_match_bruteforce(slot_priority, fallback):
+    for seed, (T, N, k, cf) in enumerate([(37, 5, 2, 0.9), (50, 8, 3, 1.0), (64, 4, 1, 0.5),
+                                          (20, 3, 3, 1.25)]):
+        idx = synth.synthetic_topk(100 + seed, T, N, k, skew=0.6)
+        C = int(np.floor(cf * T / N))
+        ref = oracle.dispatch(idx, N, cf, fallback=fallback, slot_priority=slot_priority)
+        want = _brute(idx, N, C, slot_priority, fallback)
+        assert ref["perm"].tolist() == want
+        inv = np.full(T * k, -1)
+        inv[np.array(want, dtype=np.int64)] = np.arange(len(want))
+        assert np.array_equal(ref["inv_row"], inv)
+        assert np.array_equal(ref["drop"], (inv < 0).astype(np.uint8))
+
+
+def test_fallback_is_drop_mode_plus_overflow_segment():
+    T, N, k, cf = 300, 16, 2, 0.75
+    idx = synth.synthetic_topk(7, T, N, k, skew=0.7)
+    drop = oracle.dispatch(idx, N, cf)
+    fb = oracle.dispatch(idx, N, cf, fallback=True)
+    assert drop["drop"].sum() > 0
+    # the routed experts' rows are unchanged; the fallback takes the dropped pairs in order
+    assert np.array_equal(fb["offsets"][:N + 1], drop["offsets"])
+    assert np.array_equal(fb["perm"][:drop["R"]], drop["perm"])
+    assert fb["perm"][drop["R"]:].tolist() == np.nonzero(drop["drop"])[0].tolist()
+    assert fb["R"] == T * k and not fb["drop"].any()
+    assert np.array_equal(fb["counts"], drop["counts"])       # f_i: pre-drop counts
+    # no capacity: nothing to re-route
+    nocap = oracle.dispatch(idx, N, 0.0, fallback=True)
+    assert nocap["offsets"][N + 1] == nocap["offsets"][N] == T * k
+    # k = 1: slot priority is token order
+    one = synth.synthetic_topk(8, T, N, 1, skew=0.7)
+    a, b = oracle.dispatch(one, N, cf), oracle.dispatch(one, N, cf, slot_priority=True)
+    assert all(np.array_equal(a[key], b[key]) for key in ("perm", "inv_row", "drop", "offsets"))
+
+
+def test_fallback_layer_adds_the_fallback_expert_for_dropped_slots():
+    # y(fallback) = y(drop) + sum over dropped slots of g * E_N(x), E_N by numpy
+    wl = synth.Workload("fb", T=96, d=32, N=4, k=2, H=48, act="swiglu", dtype="f32",
+                        gate_mode="R", capacity_factor=0.6, overflow="fallback", seed=9)
+    host = synth.make_host(wl)
+    ref_fb = oracle.route(wl, host["x"], host["Wg"])
+    ref_dr = oracle.route(wl.with_(overflow="drop"), host["x"], host["Wg"])
+    assert ref_dr["drop"].sum() > 0
+    toks = np.arange(wl.T)
+    y_fb = oracle.forward_rows(wl, host, ref_fb, toks)
+    y_dr = oracle.forward_rows(wl.with_(overflow="drop"), host, ref_dr, toks)
+    x = oracle.decode(host["x"])
+    W1, W3, W2 = (oracle.decode(host[n])[wl.N] for n in ("W1", "W3", "W2"))
+    h = scipy.special.expit(x @ W1.T) * (x @ W1.T) * (x @ W3.T)
+    e_fb = h @ W2.T
+    dropped = ref_dr["drop"].reshape(wl.T, wl.k).astype(bool)
+    extra = (ref_dr["gate"] * dropped).sum(1)[:, None] * e_fb
+    np.testing.assert_allclose(y_fb, y_dr + extra, rtol=1e-10, atol=1e-12)
