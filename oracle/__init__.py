@@ -143,6 +143,10 @@ def dispatch(idx: np.ndarray, N: int, capacity_factor: float, fallback: bool = F
     ("moe communication costs", Capacity factor and token dropping)."""
     idx = _c(idx.astype(np.int32))
     T, k = idx.shape
+    # the capacity factor is the fp32 value a layer configuration carries:
+    # C = floor(cf * T / N) with cf rounded to fp32 (e.g. 0.7 -> 0.69999999,
+    # so 0.7 * 400 / 8 gives C = 34)
+    capacity_factor = float(np.float32(capacity_factor))
     counts = np.empty(N, np.int32)
     kept = np.empty(N, np.int32)
     offsets = np.empty(N + 2 if fallback else N + 1, np.int32)

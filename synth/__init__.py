@@ -126,7 +126,8 @@ class Workload:
         """C = floor(capacity_factor * T / N), or -1 when unlimited (page 5)."""
         if self.capacity_factor <= 0:
             return -1
-        return int(math.floor(self.capacity_factor * self.T / self.N))
+        # the factor as the fp32 value the layer configuration carries
+        return int(math.floor(float(np.float32(self.capacity_factor)) * self.T / self.N))
 
 
 # The five workloads.  Names say what they are shaped like.

@@ -161,7 +161,7 @@ def test_capacity_variants_match_bruteforce(slot_priority, fallback):
     for seed, (T, N, k, cf) in enumerate([(37, 5, 2, 0.9), (50, 8, 3, 1.0), (64, 4, 1, 0.5),
                                           (20, 3, 3, 1.25)]):
         idx = synth.synthetic_topk(100 + seed, T, N, k, skew=0.6)
-        C = int(np.floor(cf * T / N))
+        C = int(np.floor(float(np.float32(cf)) * T / N))
         ref = oracle.dispatch(idx, N, cf, fallback=fallback, slot_priority=slot_priority)
         want = _brute(idx, N, C, slot_priority, fallback)
         assert ref["perm"].tolist() == want
@@ -210,3 +210,16 @@ def test_fallback_layer_adds_the_fallback_expert_for_dropped_slots():
     dropped = ref_dr["drop"].reshape(wl.T, wl.k).astype(bool)
     extra = (ref_dr["gate"] * dropped).sum(1)[:, None] * e_fb
     np.testing.assert_allclose(y_fb, y_dr + extra, rtol=1e-10, atol=1e-12)
+
+
+def test_capacity_uses_the_fp32_capacity_factor():
+    # the layer configuration carries the capacity factor in fp32; 0.7 rounds to
+    # 0.699999988, so with T = 400 and N = 8, C = floor(34.9999994) = 34, not 35
+    assert float(np.float32(0.7)) * 400 / 8 < 35.0
+    wl = synth.Workload("c", T=400, d=8, N=8, k=1, H=8, act="relu", dtype="f32", gate_mode="R",
+                        capacity_factor=0.7)
+    assert wl.capacity() == 34
+    idx = np.zeros((400, 1), np.int32)                 # every token on expert 0
+    ref = oracle.dispatch(idx, 8, 0.7)
+    assert ref["kept"][0] == 34 and ref["R"] == 34
+    assert oracle.dispatch(idx, 8, 0.75)["kept"][0] == 37    # exact in fp32: floor(37.5)
