@@ -295,6 +295,8 @@ def config_of(wl):
          "act": wl.act, "gate_mode": wl.gate_mode, "renormalize": wl.renormalize,
          "capacity_factor": wl.capacity_factor, "H_shared": wl.H_shared,
          "dispatch": wl.dispatch_dtype, "seed": wl.seed,
+         "n_groups": wl.n_groups, "topk_groups": wl.topk_groups, "overflow": wl.overflow,
+         "slot_priority": wl.slot_priority,
          "l2": "inputs larger than L2: expert weights read every step exceed 126 MB and the "
                "token batch rotates over 4 resident copies"}
     return c
@@ -373,7 +375,10 @@ def run_ours(args, wl):
         torch.cuda.synchronize()
         kept = counts.cpu().numpy().astype(np.int64)
         if wl.capacity_factor > 0:
+            over = int((kept - np.minimum(kept, wl.capacity())).sum())
             kept = np.minimum(kept, wl.capacity())
+            if wl.overflow == "fallback":
+                kept = np.append(kept, over)      # the fallback expert's rows
         kept_steps.append(kept)
 
     # ---- timed region (device events, max over ranks).  Nothing but the

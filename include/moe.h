@@ -84,6 +84,17 @@ enum { MOE_GATE_TOPK_THEN_SOFTMAX = 0, MOE_GATE_SOFTMAX_THEN_TOPK = 1 };
  *                   SwiGLU: y = (silu(x W1) * (x W3)) W2, silu(a) = a / (1 + e^-a). */
 enum { MOE_ACT_RELU = 0, MOE_ACT_SWIGLU = 1 };
 
+/* What happens to (token, slot) pairs an expert cannot take under its
+ * capacity C ("moe communication costs", Capacity factor and token dropping:
+ * overflowing tokens are either dropped or re-routed to a shared fallback
+ * expert).
+ *  MOE_OVERFLOW_DROP: dropped (they contribute nothing).
+ *  MOE_OVERFLOW_FALLBACK: re-routed, with their gate weight, to a fallback
+ *    expert stored as expert N after the routed ones (W1, W3, W2 then hold
+ *    N + 1 expert blocks); it has no capacity limit and takes the overflow of
+ *    every expert in the order the pairs are taken. */
+enum { MOE_OVERFLOW_DROP = 0, MOE_OVERFLOW_FALLBACK = 1 };
+
 typedef struct moe_config {
     int64_t T;               /* tokens, >= 0 */
     int32_t d;               /* hidden size; multiple of 8 (bf16) or 4 (f32) */
@@ -112,6 +123,10 @@ typedef struct moe_config {
      * still use the softmax over all N.  0 / 0: no nodes. */
     int32_t n_groups;
     int32_t topk_groups;
+    int32_t overflow;        /* MOE_OVERFLOW_*; only matters with a capacity limit */
+    int32_t slot_priority;   /* 0: capacity is filled token by token (t, then slot j);
+                              * 1: slot by slot, every token's first choice before any
+                              * token's second (priority for the top choices when k > 1) */
 } moe_config;
 
 /* Bytes of workspace every entry point below needs for `cfg` (0 on an invalid
@@ -141,19 +156,22 @@ moe_status moe_router(const moe_config *cfg, const void *x, const void *Wg, cons
  *   x             [T, d] dtype
  *   topk_idx      [T, k] int32, values in [0, N) and distinct per token
  *   expert_counts [N] int32 out: pairs routed to each expert before dropping
- *   expert_offsets[N+1] int32 out: exclusive prefix sum of min(count, C)
+ *   expert_offsets[N+1] int32 out: exclusive prefix sum of min(count, C); with
+ *                 MOE_OVERFLOW_FALLBACK [N+2], the fallback expert's rows being
+ *                 [offsets[N], offsets[N+1]) (R = offsets[N+1] = the pairs kept)
  *   perm          [T*k] int32 out: perm[row] = t*k + j for rows < R = offsets[N]
  *   inv_row       [T*k] int32 out: row of pair (t, j), or -1 if dropped
- *   drop_mask     [T*k] uint8 out: 1 if dropped
+ *   drop_mask     [T*k] uint8 out: 1 if dropped (never with the fallback expert)
  *   x_perm        [T*k, d] out: row r = x[perm[r] / k]; dispatch_dtype
  *                 (FP8: E4M3 codes, one byte each)
  *   x_scale       [T*k] fp32 out for FP8 dispatch (per-token amax / 448), else NULL
  *   p_mean        [N] fp32 in (from moe_router) or NULL
  *   f             [N] fp32 out or NULL: count / (T*k)
  *   aux_loss      [1] fp32 out or NULL (needs p_mean): alpha * N * sum f_i p_mean_i
- * Within an expert, pairs are ordered by token index; when an expert gets more
- * than C pairs the first C in token order are kept.  Rows >= R of perm and
- * x_perm are left untouched. */
+ * Within an expert, pairs are ordered by token index (slot_priority: by slot,
+ * then token); when an expert gets more than C pairs the first C in that order
+ * are kept, the rest dropped or (fallback) appended to the fallback expert's
+ * rows in the same order.  Rows >= R of perm and x_perm are left untouched. */
 moe_status moe_dispatch(const moe_config *cfg, const void *x, const int32_t *topk_idx,
                         int32_t *expert_counts, int32_t *expert_offsets, int32_t *perm,
                         int32_t *inv_row, uint8_t *drop_mask, void *x_perm, float *x_scale,
@@ -191,7 +209,8 @@ moe_status moe_dispatch_noalloc(const moe_config *cfg, const void *x, const int3
  * serve", Expert parallelism step 2).
  *   x_perm         [T*k, d] dispatch_dtype (rows >= offsets[N] are ignored)
  *   x_scale        [T*k] fp32 for FP8 dispatch, else NULL
- *   expert_offsets [N+1] int32 (device), segment e = rows [offsets[e], offsets[e+1])
+ *   expert_offsets [N+1] int32 (device), segment e = rows [offsets[e], offsets[e+1]);
+ *                  [N+2] with MOE_OVERFLOW_FALLBACK (expert N = the fallback)
  *   W1, W3, W2     stacked expert weights (W3 NULL for ReLU)
  *   y_perm         [T*k, d] dtype out; rows >= offsets[N] untouched
  * The hidden activations live in the workspace (bf16 for bf16 layers). */

@@ -18,7 +18,8 @@ def cfg_of(wl: synth.Workload) -> moe.moe_config:
                            capacity_factor=wl.capacity_factor, gate_mode=wl.gate_mode,
                            renormalize=wl.renormalize, act=wl.act, dtype=wl.dtype,
                            dispatch_dtype=wl.dispatch or None, aux_alpha=wl.aux_alpha,
-                           n_groups=wl.n_groups, topk_groups=wl.topk_groups)
+                           n_groups=wl.n_groups, topk_groups=wl.topk_groups,
+                           overflow=wl.overflow, slot_priority=wl.slot_priority)
 
 
 def tdtype(wl: synth.Workload):

@@ -108,4 +108,4 @@ def test_node_limited_config_validation(lib):
         assert moe.moe_workspace_bytes(moe.make_config(**{**ok, **bad})) == 0, bad
     # the C struct and its ctypes mirror agree on the appended fields
     import ctypes
-    assert ctypes.sizeof(moe.moe_config) == 64
+    assert ctypes.sizeof(moe.moe_config) == 72

@@ -76,7 +76,8 @@ def test_layer_deterministic(name):
 
 FULL = {"tiny": (synth.TINY_F32, 256), "mixtral": (synth.MIXTRAL, 48),
         "switch": (synth.SWITCH, 512), "deepseek": (synth.DEEPSEEK, 12),
-        "grok": (synth.GROK, 32), "deepseek-nl": (synth.DEEPSEEK_NODE_LIMITED, 12)}
+        "grok": (synth.GROK, 32), "deepseek-nl": (synth.DEEPSEEK_NODE_LIMITED, 12),
+        "switch-fb": (synth.SWITCH_FALLBACK, 512)}
 
 
 @pytest.mark.slow

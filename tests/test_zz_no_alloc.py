@@ -29,6 +29,8 @@ CASES = {
     "capacity-bf16": synth.SWITCH.with_(T=1000, d=128, H=256),
     "fp8-k8": synth.DEEPSEEK.with_(T=200, d=256, H=128, H_shared=128),
     "fp32": synth.TINY_F32,
+    "fallback-slot": synth.MIXTRAL.with_(T=600, d=128, N=8, H=256, capacity_factor=0.7,
+                                         overflow="fallback", slot_priority=True),
 }
 
 
@@ -37,7 +39,7 @@ def _buffers(wl):
     fp8 = wl.dispatch == "fp8"
     return dict(
         counts=torch.empty(wl.N, dtype=torch.int32, device="cuda"),
-        offs=torch.empty(wl.N + 1, dtype=torch.int32, device="cuda"),
+        offs=torch.empty(wl.N + 2, dtype=torch.int32, device="cuda"),
         perm=torch.full((rows,), -1, dtype=torch.int32, device="cuda"),
         inv=torch.empty(rows, dtype=torch.int32, device="cuda"),
         drop=torch.empty(rows, dtype=torch.uint8, device="cuda"),
@@ -45,12 +47,14 @@ def _buffers(wl):
         xs=torch.zeros(rows, dtype=torch.float32, device="cuda") if fp8 else None,
         f=torch.empty(wl.N, dtype=torch.float32, device="cuda"),
         aux=torch.empty(1, dtype=torch.float32, device="cuda"),
+        n_off=wl.N + (2 if wl.overflow == "fallback" else 1),
     )
 
 
 def _same(a, b, R):
     assert torch.equal(a["counts"], b["counts"])
-    assert torch.equal(a["offs"], b["offs"])
+    n = a["n_off"]
+    assert torch.equal(a["offs"][:n], b["offs"][:n])
     assert torch.equal(a["perm"][:R], b["perm"][:R])
     assert torch.equal(a["inv"], b["inv"])
     assert torch.equal(a["drop"], b["drop"])
@@ -79,7 +83,7 @@ def test_noalloc_dispatch_matches_workspace_dispatch(name):
                                  got["aux"])
         torch.cuda.synchronize()
         assert moe.moe_check_status(ws)[0] == moe.MOE_OK
-        R = int(ref["offs"][-1].item())
+        R = int(ref["offs"][ref["n_off"] - 1].item())
         _same(ref, got, R)
 
 

@@ -23,6 +23,7 @@ MOE_ERR_CUDA, MOE_ERR_DEVICE_STATUS, MOE_ERR_TIMEOUT = 4, 5, 6
 MOE_F32, MOE_BF16, MOE_FP8_E4M3 = 0, 1, 2
 MOE_GATE_TOPK_THEN_SOFTMAX, MOE_GATE_SOFTMAX_THEN_TOPK = 0, 1
 MOE_ACT_RELU, MOE_ACT_SWIGLU = 0, 1
+MOE_OVERFLOW_DROP, MOE_OVERFLOW_FALLBACK = 0, 1
 
 EXPORTS = ("moe_workspace_bytes", "moe_router", "moe_dispatch", "moe_expert_ffn", "moe_combine",
            "moe_layer_forward", "moe_check_status", "moe_status_string", "moe_last_error_string",
@@ -39,7 +40,8 @@ class moe_config(ctypes.Structure):
                 ("renormalize", ctypes.c_int32), ("act", ctypes.c_int32),
                 ("dtype", ctypes.c_int32), ("dispatch_dtype", ctypes.c_int32),
                 ("aux_alpha", ctypes.c_float), ("n_groups", ctypes.c_int32),
-                ("topk_groups", ctypes.c_int32)]
+                ("topk_groups", ctypes.c_int32), ("overflow", ctypes.c_int32),
+                ("slot_priority", ctypes.c_int32)]
 
 
 class MoeError(RuntimeError):
@@ -133,14 +135,17 @@ def _check(status: int, where: str):
 
 def make_config(T, d, N, k, H, *, H_shared=0, capacity_factor=0.0, gate_mode="R",
                 renormalize=False, act="swiglu", dtype="bf16", dispatch_dtype=None,
-                aux_alpha=0.01, n_groups=0, topk_groups=0) -> moe_config:
+                aux_alpha=0.01, n_groups=0, topk_groups=0, overflow="drop",
+                slot_priority=False) -> moe_config:
     dt = {"f32": MOE_F32, "bf16": MOE_BF16}[dtype]
     dd = dt if dispatch_dtype in (None, "", dtype) else {"fp8": MOE_FP8_E4M3}[dispatch_dtype]
     return moe_config(int(T), int(d), int(N), int(k), int(H), int(H_shared),
                       float(capacity_factor),
                       MOE_GATE_TOPK_THEN_SOFTMAX if gate_mode == "R" else MOE_GATE_SOFTMAX_THEN_TOPK,
                       int(bool(renormalize)), MOE_ACT_RELU if act == "relu" else MOE_ACT_SWIGLU,
-                      dt, dd, float(aux_alpha), int(n_groups), int(topk_groups))
+                      dt, dd, float(aux_alpha), int(n_groups), int(topk_groups),
+                      {"drop": MOE_OVERFLOW_DROP, "fallback": MOE_OVERFLOW_FALLBACK}[overflow],
+                      int(bool(slot_priority)))
 
 
 def moe_workspace_bytes(cfg: moe_config) -> int:

@@ -37,9 +37,16 @@ constexpr int kThreads = 256;
 constexpr int kWarps = kThreads / 32;
 constexpr int kPerWarp = kDispChunk / kWarps;  // 256 pairs, 8 rounds of 32
 
+// Pair index at position p of the order in which pairs are taken: token by
+// token (p itself), or slot by slot (every token's first choice first).
+__device__ __forceinline__ int64_t pair_at(int64_t p, int64_t T, int k, int slot_priority)
+{
+    return slot_priority ? (p % T) * k + p / T : p;
+}
+
 __global__ void __launch_bounds__(kThreads)
-    dispatch_count_kernel(const int32_t *__restrict__ idx, int64_t n_pairs, int N,
-                          int32_t *__restrict__ block_base, uint32_t *status)
+    dispatch_count_kernel(const int32_t *__restrict__ idx, int64_t T, int k, int slot_priority,
+                          int N, int32_t *__restrict__ block_base, uint32_t *status)
 {
     grid_dep_wait();
     extern __shared__ int32_t s_cnt[];
@@ -47,12 +54,13 @@ __global__ void __launch_bounds__(kThreads)
         s_cnt[e] = 0;
     __syncthreads();
     const int lane = threadIdx.x & 31;
+    const int64_t n_pairs = T * k;
     const int64_t base = static_cast<int64_t>(blockIdx.x) * kDispChunk;
     for (int r = 0; r < kDispChunk / kThreads; ++r) {
-        const int64_t i = base + r * kThreads + threadIdx.x;
+        const int64_t p = base + r * kThreads + threadIdx.x;
         int e = -1;
-        if (i < n_pairs) {
-            e = idx[i];
+        if (p < n_pairs) {
+            e = idx[pair_at(p, T, k, slot_priority)];
             if (e < 0 || e >= N) {
                 set_status(status, DEV_BAD_EXPERT);
                 e = -1;
@@ -69,10 +77,13 @@ __global__ void __launch_bounds__(kThreads)
 
 // Per expert e (thread e of a 1024-thread block, e < N): total count `run`,
 // kept = min(run, C), offsets = exclusive scan of kept over experts, f and
-// L_aux = alpha N sum_e f_e p_e summed in a fixed tree order.  Also leaves
-// offsets in s_off when it is given.  Every thread of the block calls it.
+// L_aux = alpha N sum_e f_e p_e summed in a fixed tree order; with a fallback
+// expert also offsets[N + 1] = offsets[N] + the pairs over capacity.  Also
+// leaves offsets[0..N] in s_off when it is given.  Every thread of the block
+// calls it.
 __device__ __forceinline__ void expert_offsets_and_aux(int e, int32_t run, int N, int64_t n_pairs,
-                                                       int64_t C, int32_t *__restrict__ counts,
+                                                       int64_t C, int fallback,
+                                                       int32_t *__restrict__ counts,
                                                        int32_t *__restrict__ offsets,
                                                        const float *__restrict__ p_mean,
                                                        float *__restrict__ f,
@@ -80,6 +91,7 @@ __device__ __forceinline__ void expert_offsets_and_aux(int e, int32_t run, int N
                                                        int32_t *s_off)
 {
     __shared__ int32_t s_warp[32];
+    __shared__ int32_t s_over[32];
     __shared__ double s_aux[1024];
     const int lane = e & 31, warp = e >> 5;
     int32_t kept = 0;
@@ -89,27 +101,35 @@ __device__ __forceinline__ void expert_offsets_and_aux(int e, int32_t run, int N
         if (f != nullptr)
             f[e] = static_cast<float>(static_cast<double>(run) / static_cast<double>(n_pairs));
     }
-    // exclusive scan of kept over experts
+    // exclusive scan of kept over experts; sum of the overflow
     int32_t incl = kept;
+    int32_t over = run - kept;
 #pragma unroll
     for (int o = 1; o < 32; o <<= 1) {
         const int32_t v = __shfl_up_sync(0xffffffffu, incl, o);
         if (lane >= o)
             incl += v;
+        over += __shfl_xor_sync(0xffffffffu, over, o);
     }
     if (lane == 31)
         s_warp[warp] = incl;
+    if (lane == 0)
+        s_over[warp] = over;
     __syncthreads();
     if (warp == 0) {
         int32_t w = s_warp[lane];
         int32_t wi = w;
+        int32_t ov = s_over[lane];
 #pragma unroll
         for (int o = 1; o < 32; o <<= 1) {
             const int32_t v = __shfl_up_sync(0xffffffffu, wi, o);
             if (lane >= o)
                 wi += v;
+            ov += __shfl_xor_sync(0xffffffffu, ov, o);
         }
         s_warp[lane] = wi - w;  // exclusive warp base
+        if (lane == 0)
+            s_over[0] = ov;
     }
     __syncthreads();
     const int32_t excl = s_warp[warp] + incl - kept;
@@ -118,8 +138,13 @@ __device__ __forceinline__ void expert_offsets_and_aux(int e, int32_t run, int N
         if (s_off != nullptr)
             s_off[e] = excl;
     }
-    if (e == N - 1)
+    if (e == N - 1) {
         offsets[N] = excl + kept;
+        if (s_off != nullptr)
+            s_off[N] = excl + kept;
+        if (fallback)
+            offsets[N + 1] = excl + kept + s_over[0];
+    }
     // L_aux = alpha N sum_e f_e p_e, summed in a fixed tree order
     if (aux_loss != nullptr && p_mean != nullptr) {
         double term = 0.0;
@@ -138,54 +163,118 @@ __device__ __forceinline__ void expert_offsets_and_aux(int e, int32_t run, int N
     }
 }
 
+// Exclusive prefix sum of v[0..n) in place by one 1024-thread block.
+__device__ void block_exclusive_scan(int32_t *v, int n)
+{
+    __shared__ int32_t s_part[32];
+    __shared__ int32_t s_carry;
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    if (threadIdx.x == 0)
+        s_carry = 0;
+    __syncthreads();
+    for (int c0 = 0; c0 < n; c0 += 1024) {
+        const int i = c0 + static_cast<int>(threadIdx.x);
+        const int32_t x = i < n ? v[i] : 0;
+        int32_t incl = x;
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+            const int32_t y = __shfl_up_sync(0xffffffffu, incl, o);
+            if (lane >= o)
+                incl += y;
+        }
+        if (lane == 31)
+            s_part[warp] = incl;
+        __syncthreads();
+        if (warp == 0) {
+            const int32_t w = s_part[lane];
+            int32_t wi = w;
+#pragma unroll
+            for (int o = 1; o < 32; o <<= 1) {
+                const int32_t y = __shfl_up_sync(0xffffffffu, wi, o);
+                if (lane >= o)
+                    wi += y;
+            }
+            s_part[lane] = wi - w;
+        }
+        __syncthreads();
+        const int32_t carry = s_carry;
+        if (i < n)
+            v[i] = carry + s_part[warp] + incl - x;
+        __syncthreads();
+        if (threadIdx.x == 1023)
+            s_carry = carry + s_part[31] + incl;
+        __syncthreads();
+    }
+}
+
 __global__ void __launch_bounds__(1024)
-    dispatch_scan_kernel(int nblk, int N, int64_t n_pairs, int64_t C,
+    dispatch_scan_kernel(int nblk, int N, int64_t n_pairs, int64_t C, int fallback,
                          int32_t *__restrict__ block_base, int32_t *__restrict__ counts,
                          int32_t *__restrict__ offsets, const float *__restrict__ p_mean,
                          float *__restrict__ f, float *__restrict__ aux_loss, float alpha)
 {
     grid_dep_wait();
     const int e = threadIdx.x;
+    // fallback: pairs of block b over capacity, then their exclusive scan
+    int32_t *fb_base = block_base + static_cast<int64_t>(nblk) * N;
+    const bool fb = fallback && C >= 0;
+    if (fb)
+        for (int b = threadIdx.x; b < nblk; b += 1024)
+            fb_base[b] = 0;
+    __syncthreads();
     int32_t run = 0;
     if (e < N) {
         for (int b = 0; b < nblk; ++b) {
             const int64_t o = static_cast<int64_t>(b) * N + e;
             const int32_t v = block_base[o];
             block_base[o] = run;
+            if (fb) {
+                // pairs of this block past the first C of the expert
+                int64_t over = static_cast<int64_t>(run) + v - C;
+                over = over < 0 ? 0 : (over > v ? v : over);
+                if (over > 0)
+                    atomicAdd(&fb_base[b], static_cast<int32_t>(over));
+            }
             run += v;
         }
     }
-    expert_offsets_and_aux(e, run, N, n_pairs, C, counts, offsets, p_mean, f, aux_loss, alpha,
-                           nullptr);
+    __syncthreads();
+    if (fb)
+        block_exclusive_scan(fb_base, nblk);
+    expert_offsets_and_aux(e, run, N, n_pairs, C, fallback, counts, offsets, p_mean, f, aux_loss,
+                           alpha, nullptr);
 }
 
 // The whole sort in one block, for batches of at most kFusedMaxPairs pairs and
 // N <= kFusedMaxN experts: each of the 32 warps takes a contiguous range of
-// pairs (in pair order), counts its experts, a column scan over the warps
-// gives every warp its base inside each expert, and a second walk over the
-// range (expert ids kept in shared memory) ranks each pair stably.  Same
-// results as count + scan + rank, in one launch without a workspace.
+// positions (in the order pairs are taken), counts its experts, a column scan
+// over the warps gives every warp its base inside each expert, and a second
+// walk (expert ids kept in shared memory) ranks each pair stably; with a
+// fallback expert a third walk places the pairs over capacity.  Same results
+// as count + scan + rank, in one launch without a workspace.
 constexpr int kFusedThreads = 1024;
 constexpr int kFusedWarps = kFusedThreads / 32;
 
 __global__ void __launch_bounds__(kFusedThreads)
-    dispatch_fused_kernel(const int32_t *__restrict__ idx, int64_t n_pairs, int N, int64_t C,
-                          int32_t *__restrict__ counts, int32_t *__restrict__ offsets,
-                          int32_t *__restrict__ perm, int32_t *__restrict__ inv_row,
-                          uint8_t *__restrict__ drop, const float *__restrict__ p_mean,
-                          float *__restrict__ f, float *__restrict__ aux_loss, float alpha,
-                          uint32_t *status)
+    dispatch_fused_kernel(const int32_t *__restrict__ idx, int64_t T, int k, int slot_priority,
+                          int N, int64_t C, int fallback, int32_t *__restrict__ counts,
+                          int32_t *__restrict__ offsets, int32_t *__restrict__ perm,
+                          int32_t *__restrict__ inv_row, uint8_t *__restrict__ drop,
+                          const float *__restrict__ p_mean, float *__restrict__ f,
+                          float *__restrict__ aux_loss, float alpha, uint32_t *status)
 {
     grid_dep_wait();
     extern __shared__ int32_t s_fz[];
     int32_t *s_cnt = s_fz;                                              // [32][N]
-    int16_t *s_e = reinterpret_cast<int16_t *>(s_fz + kFusedWarps * N);  // [n_pairs]
-    __shared__ int32_t s_off[kFusedMaxN];
+    int16_t *s_e = reinterpret_cast<int16_t *>(s_fz + kFusedWarps * N);  // [n_pairs], by position
+    __shared__ int32_t s_off[kFusedMaxN + 1];
+    __shared__ int32_t s_fbw[kFusedWarps];
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int64_t n_pairs = T * k;
     for (int i = threadIdx.x; i < kFusedWarps * N; i += kFusedThreads)
         s_cnt[i] = 0;
     __syncthreads();
-    // pairs per warp, a multiple of 32
+    // positions per warp, a multiple of 32
     const int64_t per_w = (n_pairs + 32 * kFusedWarps - 1) / (32 * kFusedWarps) * 32;
     const int64_t wb = warp * per_w;
     int32_t *mine = s_cnt + warp * N;
@@ -194,21 +283,22 @@ __global__ void __launch_bounds__(kFusedThreads)
         int ev[U];
 #pragma unroll
         for (int u = 0; u < U; ++u) {
-            const int64_t i = wb + r0 + 32 * u + lane;
-            ev[u] = (r0 + 32 * u < per_w && i < n_pairs) ? idx[i] : -1;
+            const int64_t p = wb + r0 + 32 * u + lane;
+            ev[u] = (r0 + 32 * u < per_w && p < n_pairs) ? idx[pair_at(p, T, k, slot_priority)]
+                                                         : -1;
         }
 #pragma unroll
         for (int u = 0; u < U; ++u) {
             if (r0 + 32 * u >= per_w)
                 break;
-            const int64_t i = wb + r0 + 32 * u + lane;
+            const int64_t p = wb + r0 + 32 * u + lane;
             int e = ev[u];
-            if (i < n_pairs) {
+            if (p < n_pairs) {
                 if (e < 0 || e >= N) {
                     set_status(status, DEV_BAD_EXPERT);
                     e = -1;
                 }
-                s_e[i] = static_cast<int16_t>(e);
+                s_e[p] = static_cast<int16_t>(e);
             }
             const uint32_t peers = __match_any_sync(0xffffffffu, e);
             if (e >= 0 && lane == __ffs(peers) - 1)
@@ -227,13 +317,14 @@ __global__ void __launch_bounds__(kFusedThreads)
             run += v;
         }
     }
-    expert_offsets_and_aux(threadIdx.x, run, N, n_pairs, C, counts, offsets, p_mean, f, aux_loss,
-                           alpha, s_off);
+    expert_offsets_and_aux(threadIdx.x, run, N, n_pairs, C, fallback, counts, offsets, p_mean, f,
+                           aux_loss, alpha, s_off);
     __syncthreads();
     // walk again in order; rank = warp base + earlier rounds + earlier lanes
+    int32_t n_over = 0;   // this warp's pairs over capacity (fallback)
     for (int64_t r = 0; r < per_w; r += 32) {
-        const int64_t i = wb + r + lane;
-        const int e = i < n_pairs ? static_cast<int>(s_e[i]) : -1;
+        const int64_t p = wb + r + lane;
+        const int e = p < n_pairs ? static_cast<int>(s_e[p]) : -1;
         const uint32_t peers = __match_any_sync(0xffffffffu, e);
         int32_t rank = 0;
         if (e >= 0)
@@ -242,10 +333,15 @@ __global__ void __launch_bounds__(kFusedThreads)
         if (e >= 0 && lane == __ffs(peers) - 1)
             mine[e] += __popc(peers);
         __syncwarp();
-        if (i < n_pairs) {
-            if (e < 0 || (C >= 0 && rank >= C)) {
+        const bool over = e >= 0 && C >= 0 && rank >= C;
+        n_over += __popc(__ballot_sync(0xffffffffu, over && fallback));
+        if (p < n_pairs) {
+            const int64_t i = pair_at(p, T, k, slot_priority);
+            if (e < 0 || (over && !fallback)) {
                 drop[i] = 1;
                 inv_row[i] = -1;
+            } else if (over) {
+                s_e[p] = -2;   // placed by the walk below
             } else {
                 const int32_t row = s_off[e] + rank;
                 perm[row] = static_cast<int32_t>(i);
@@ -254,17 +350,53 @@ __global__ void __launch_bounds__(kFusedThreads)
             }
         }
     }
+    if (!fallback)
+        return;
+    // fallback rows: offsets[N] + the overflow of earlier warps + earlier rounds and lanes
+    if (lane == 0)
+        s_fbw[warp] = n_over;
+    __syncthreads();
+    if (warp == 0) {
+        const int32_t w = s_fbw[lane];
+        int32_t wi = w;
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+            const int32_t y = __shfl_up_sync(0xffffffffu, wi, o);
+            if (lane >= o)
+                wi += y;
+        }
+        s_fbw[lane] = wi - w;
+    }
+    __syncthreads();
+    int32_t pos = s_off[N] + s_fbw[warp];
+    for (int64_t r = 0; r < per_w; r += 32) {
+        const int64_t p = wb + r + lane;
+        const bool mark = p < n_pairs && s_e[p] == -2;
+        const uint32_t bal = __ballot_sync(0xffffffffu, mark);
+        if (mark) {
+            const int64_t i = pair_at(p, T, k, slot_priority);
+            const int32_t row = pos + __popc(bal & lanemask_lt());
+            perm[row] = static_cast<int32_t>(i);
+            inv_row[i] = row;
+            drop[i] = 0;
+        }
+        pos += __popc(bal);
+    }
 }
 
 __global__ void __launch_bounds__(kThreads)
-    dispatch_rank_kernel(const int32_t *__restrict__ idx, int64_t n_pairs, int N, int64_t C,
-                         const int32_t *__restrict__ block_base,
+    dispatch_rank_kernel(const int32_t *__restrict__ idx, int64_t T, int k, int slot_priority,
+                         int N, int64_t C, int fallback, const int32_t *__restrict__ block_base,
                          const int32_t *__restrict__ offsets, int32_t *__restrict__ perm,
                          int32_t *__restrict__ inv_row, uint8_t *__restrict__ drop)
 {
     grid_dep_wait();
     extern __shared__ int32_t s_w[];  // [kWarps][N]
+    __shared__ uint8_t s_over[kDispChunk];   // fallback: position over capacity
+    __shared__ int32_t s_fbw[kWarps];
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int64_t n_pairs = T * k;
+    const int nblk = static_cast<int>((n_pairs + kDispChunk - 1) / kDispChunk);
     for (int i = threadIdx.x; i < kWarps * N; i += kThreads)
         s_w[i] = 0;
     __syncthreads();
@@ -272,10 +404,10 @@ __global__ void __launch_bounds__(kThreads)
     int32_t *mine = s_w + warp * N;
     // phase 1: per-warp counts
     for (int r = 0; r < kPerWarp / 32; ++r) {
-        const int64_t i = wbase + r * 32 + lane;
+        const int64_t p = wbase + r * 32 + lane;
         int e = -1;
-        if (i < n_pairs) {
-            e = idx[i];
+        if (p < n_pairs) {
+            e = idx[pair_at(p, T, k, slot_priority)];
             if (e < 0 || e >= N)
                 e = -1;
         }
@@ -296,11 +428,12 @@ __global__ void __launch_bounds__(kThreads)
     }
     __syncthreads();
     // phase 3: walk the pairs in order; rank = warp base + earlier lanes
+    int32_t n_over = 0;
     for (int r = 0; r < kPerWarp / 32; ++r) {
-        const int64_t i = wbase + r * 32 + lane;
+        const int64_t p = wbase + r * 32 + lane;
         int e = -1;
-        if (i < n_pairs) {
-            e = idx[i];
+        if (p < n_pairs) {
+            e = idx[pair_at(p, T, k, slot_priority)];
             if (e < 0 || e >= N)
                 e = -1;
         }
@@ -312,17 +445,51 @@ __global__ void __launch_bounds__(kThreads)
         if (e >= 0 && lane == __ffs(peers) - 1)
             mine[e] += __popc(peers);
         __syncwarp();
-        if (i < n_pairs) {
-            if (e < 0 || (C >= 0 && rank >= C)) {
+        const bool over = e >= 0 && C >= 0 && rank >= C;
+        n_over += __popc(__ballot_sync(0xffffffffu, over && fallback));
+        s_over[warp * kPerWarp + r * 32 + lane] = (over && fallback) ? 1 : 0;
+        if (p < n_pairs) {
+            const int64_t i = pair_at(p, T, k, slot_priority);
+            if (e < 0 || (over && !fallback)) {
                 drop[i] = 1;
                 inv_row[i] = -1;
-            } else {
+            } else if (!over) {
                 const int32_t row = offsets[e] + rank;
                 perm[row] = static_cast<int32_t>(i);
                 inv_row[i] = row;
                 drop[i] = 0;
             }
         }
+    }
+    if (!fallback)
+        return;
+    // phase 4 (fallback): this block's pairs over capacity, in order, after
+    // those of earlier blocks (scan kernel) and earlier warps
+    if (lane == 0)
+        s_fbw[warp] = n_over;
+    __syncthreads();
+    if (threadIdx.x == 0) {
+        int32_t run = offsets[N] + block_base[static_cast<int64_t>(nblk) * N + blockIdx.x];
+        for (int w = 0; w < kWarps; ++w) {
+            const int32_t v = s_fbw[w];
+            s_fbw[w] = run;
+            run += v;
+        }
+    }
+    __syncthreads();
+    int32_t pos = s_fbw[warp];
+    for (int r = 0; r < kPerWarp / 32; ++r) {
+        const int64_t p = wbase + r * 32 + lane;
+        const bool mark = s_over[warp * kPerWarp + r * 32 + lane] != 0;
+        const uint32_t bal = __ballot_sync(0xffffffffu, mark);
+        if (mark) {
+            const int64_t i = pair_at(p, T, k, slot_priority);
+            const int32_t row = pos + __popc(bal & lanemask_lt());
+            perm[row] = static_cast<int32_t>(i);
+            inv_row[i] = row;
+            drop[i] = 0;
+        }
+        pos += __popc(bal);
     }
 }
 
@@ -530,19 +697,20 @@ cudaError_t launch_dispatch(const DispatchLaunch &L, cudaStream_t stream)
                 return err;
             attr_set = true;
         }
-        launch_k(dispatch_fused_kernel, 1, kFusedThreads, smem, stream, L.topk_idx, n_pairs, L.N,
-                 L.capacity, L.counts, L.offsets, L.perm, L.inv_row, L.drop, L.p_mean, L.f,
-                 L.aux_loss, L.aux_alpha, L.status);
+        launch_k(dispatch_fused_kernel, 1, kFusedThreads, smem, stream, L.topk_idx, L.T, L.k,
+                 L.slot_priority, L.N, L.capacity, L.fallback, L.counts, L.offsets, L.perm,
+                 L.inv_row, L.drop, L.p_mean, L.f, L.aux_loss, L.aux_alpha, L.status);
         sort_launches = 1;
     } else {
         const int nblk = static_cast<int>((n_pairs + kDispChunk - 1) / kDispChunk);
         launch_k(dispatch_count_kernel, nblk, kThreads, L.N * sizeof(int32_t), stream,
-                 L.topk_idx, n_pairs, L.N, L.block_base, L.status);
+                 L.topk_idx, L.T, L.k, L.slot_priority, L.N, L.block_base, L.status);
         launch_k(dispatch_scan_kernel, 1, 1024, 0, stream, nblk, L.N, n_pairs, L.capacity,
-                 L.block_base, L.counts, L.offsets, L.p_mean, L.f, L.aux_loss, L.aux_alpha);
+                 L.fallback, L.block_base, L.counts, L.offsets, L.p_mean, L.f, L.aux_loss,
+                 L.aux_alpha);
         launch_k(dispatch_rank_kernel, nblk, kThreads, kWarps * L.N * sizeof(int32_t), stream,
-                 L.topk_idx, n_pairs, L.N, L.capacity, L.block_base, L.offsets, L.perm,
-                 L.inv_row, L.drop);
+                 L.topk_idx, L.T, L.k, L.slot_priority, L.N, L.capacity, L.fallback, L.block_base,
+                 L.offsets, L.perm, L.inv_row, L.drop);
         sort_launches = 3;
     }
     if (L.x_perm == nullptr) {      // the caller builds the expert-ordered rows itself
@@ -554,13 +722,13 @@ cudaError_t launch_dispatch(const DispatchLaunch &L, cudaStream_t stream)
     uint8_t *xp = static_cast<uint8_t *>(L.x_perm);
     if (L.dtype == MOE_F32)
         launch_k(dispatch_gather_kernel<false, false>, grid, kThreads, 0, stream, 
-            x, L.d, L.k, L.perm, L.offsets + L.N, xp, nullptr, nullptr);
+            x, L.d, L.k, L.perm, L.offsets + L.N + (L.fallback ? 1 : 0), xp, nullptr, nullptr);
     else if (!L.fp8)
         launch_k(dispatch_gather_kernel<true, false>, grid, kThreads, 0, stream, 
-            x, L.d, L.k, L.perm, L.offsets + L.N, xp, nullptr, nullptr);
+            x, L.d, L.k, L.perm, L.offsets + L.N + (L.fallback ? 1 : 0), xp, nullptr, nullptr);
     else
         launch_k(dispatch_gather_kernel<true, true>, grid, kThreads, 0, stream, 
-            x, L.d, L.k, L.perm, L.offsets + L.N, xp, L.x_scale,
+            x, L.d, L.k, L.perm, L.offsets + L.N + (L.fallback ? 1 : 0), xp, L.x_scale,
             static_cast<__nv_bfloat16 *>(L.x_bf16_copy));
     count_launches(sort_launches + 1);
     return cudaGetLastError();

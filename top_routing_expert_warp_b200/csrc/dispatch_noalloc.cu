@@ -11,8 +11,8 @@
 // inputs and outputs.
 //
 // Limits and sharing: the array holds the counts of at most
-// kNoAllocMaxPairs (token, slot) pairs for up to 256 experts, about 128 KiB
-// per GPU, and every GPU that loads the library keeps it until the process
+// kNoAllocMaxPairs (token, slot) pairs for up to 256 experts (and the
+// fallback expert's per-block bases), about 128 KiB per GPU, and every GPU that loads the library keeps it until the process
 // exits.  All calls on a device share the one array, so calls whose work
 // overlaps on the GPU (different streams without ordering, or several host
 // threads at once) race with each other and must be serialised by the caller.
@@ -29,9 +29,10 @@ constexpr int kNoAllocMaxExperts = 256;
 constexpr int kNoAllocMaxBlocks = static_cast<int>(kNoAllocMaxPairs / moe::kDispChunk);
 constexpr int kStatusInts = 64;                 // status word, padded to 256 bytes
 
-// [0]: device status word; [kStatusInts ...]: per-block expert counts / bases.
+// [0]: device status word; [kStatusInts ...]: per-block expert counts / bases,
+// then per-block bases of the fallback expert's rows.
 static __device__ __align__(256) int32_t
-    g_noalloc_scratch[kStatusInts + kNoAllocMaxBlocks * kNoAllocMaxExperts];
+    g_noalloc_scratch[kStatusInts + kNoAllocMaxBlocks * kNoAllocMaxExperts + kNoAllocMaxBlocks];
 
 constexpr int kMaxDevices = 64;
 std::mutex g_mu;
@@ -81,9 +82,11 @@ extern "C" moe_status moe_dispatch_noalloc(const moe_config *cfg, const void *x,
         scratch = g_scratch_ptr[dev];
     }
 
+    const int fallback = cfg->overflow == MOE_OVERFLOW_FALLBACK ? 1 : 0;
     if (pairs == 0) {
         if (cudaMemsetAsync(expert_counts, 0, cfg->N * sizeof(int32_t), s) != cudaSuccess ||
-            cudaMemsetAsync(expert_offsets, 0, (cfg->N + 1) * sizeof(int32_t), s) != cudaSuccess ||
+            cudaMemsetAsync(expert_offsets, 0, (cfg->N + 1 + fallback) * sizeof(int32_t), s) !=
+                cudaSuccess ||
             (f && cudaMemsetAsync(f, 0, cfg->N * sizeof(float), s) != cudaSuccess) ||
             (aux_loss && cudaMemsetAsync(aux_loss, 0, sizeof(float), s) != cudaSuccess))
             return MOE_ERR_CUDA;
@@ -107,6 +110,8 @@ extern "C" moe_status moe_dispatch_noalloc(const moe_config *cfg, const void *x,
         D.capacity = static_cast<int64_t>(static_cast<double>(cfg->capacity_factor) *
                                           static_cast<double>(cfg->T) /
                                           static_cast<double>(cfg->N));
+    D.fallback = fallback;
+    D.slot_priority = cfg->slot_priority;
     D.topk_idx = topk_idx;
     D.block_base = scratch + kStatusInts;
     D.counts = expert_counts;

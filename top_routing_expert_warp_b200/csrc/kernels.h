@@ -126,8 +126,10 @@ struct DispatchLaunch {
     int64_t T;
     int32_t d, N, k;
     int64_t capacity;         // -1 = unlimited
+    int fallback;             // pairs over capacity go to group N (offsets has N + 2 entries)
+    int slot_priority;        // pairs taken slot by slot instead of token by token
     const int32_t *topk_idx;
-    int32_t *block_base;      // [nblk, N] workspace
+    int32_t *block_base;      // [nblk, N] workspace, then [nblk] fallback bases
     int32_t *counts;          // [N]
     int32_t *offsets;         // [N+1]
     int32_t *perm;            // [T*k]

@@ -71,6 +71,18 @@ bool node_limited(const moe_config &c)
     return c.n_groups > 1 && c.topk_groups < c.n_groups;
 }
 
+// Pairs over capacity go to the fallback expert N (one more expert group).
+bool has_fallback(const moe_config &c)
+{
+    return c.overflow == MOE_OVERFLOW_FALLBACK;
+}
+
+// Expert groups of the FFN: the routed experts, plus the fallback.
+int32_t ffn_groups(const moe_config &c)
+{
+    return c.N + (has_fallback(c) ? 1 : 0);
+}
+
 bool config_ok(const moe_config *c)
 {
     if (!c)
@@ -95,6 +107,9 @@ bool config_ok(const moe_config *c)
     if (c->T * c->k > 0x7FFFFFFFll)
         return false;
     if (c->n_groups < 0 || c->topk_groups < 0)
+        return false;
+    if ((c->overflow != MOE_OVERFLOW_DROP && c->overflow != MOE_OVERFLOW_FALLBACK) ||
+        (c->slot_priority != 0 && c->slot_priority != 1))
         return false;
     if (node_limited(*c)) {
         if (c->n_groups > 32 || c->N % c->n_groups != 0 || c->topk_groups < 1 ||
@@ -130,8 +145,8 @@ Layout layout_of(const moe_config &c)
     L.topk_w = take(rows * 4);
     L.p_mean = take(N * 4);
     L.counts = take(N * 4);
-    L.offsets = take((N + 1) * 4);
-    L.block_base = take(nblk * N * 4);
+    L.offsets = take((N + 2) * 4);
+    L.block_base = take(nblk * N * 4 + nblk * 4);   // per-block expert bases, fallback bases
     L.perm = take(rows * 4);
     L.inv_row = take(rows * 4);
     L.drop = take(rows);
@@ -250,7 +265,7 @@ moe_status run_dispatch(const moe_config &c, const void *x, const int32_t *topk_
 {
     if (c.T == 0) {
         MOE_CUDA(cudaMemsetAsync(counts, 0, c.N * sizeof(int32_t), s));
-        MOE_CUDA(cudaMemsetAsync(offsets, 0, (c.N + 1) * sizeof(int32_t), s));
+        MOE_CUDA(cudaMemsetAsync(offsets, 0, (ffn_groups(c) + 1) * sizeof(int32_t), s));
         if (f)
             MOE_CUDA(cudaMemsetAsync(f, 0, c.N * sizeof(float), s));
         if (aux_loss)
@@ -269,6 +284,8 @@ moe_status run_dispatch(const moe_config &c, const void *x, const int32_t *topk_
     if (c.capacity_factor > 0.0f)
         D.capacity = static_cast<int64_t>(static_cast<double>(c.capacity_factor) *
                                           static_cast<double>(c.T) / static_cast<double>(c.N));
+    D.fallback = has_fallback(c) ? 1 : 0;
+    D.slot_priority = c.slot_priority;
     D.topk_idx = topk_idx;
     D.block_base = w.at<int32_t>(w.L.block_base);
     D.counts = counts;
@@ -433,10 +450,12 @@ moe_status moe_expert_ffn(const moe_config *cfg, const void *x_perm, const float
     const void *A = x_perm;
     if (fp8 && rows_cap > 0) {
         MOE_CUDA(moe::launch_fp8_to_bf16(static_cast<const uint8_t *>(x_perm), rows_cap, cfg->d,
-                                         expert_offsets, cfg->N, w.at<void>(w.L.x_gemm), s));
+                                         expert_offsets, ffn_groups(*cfg), w.at<void>(w.L.x_gemm),
+                                         s));
         A = w.at<void>(w.L.x_gemm);
     }
-    return run_ffn(*cfg, A, fp8 ? x_scale : nullptr, rows_cap, expert_offsets, cfg->N, 0, cfg->H,
+    return run_ffn(*cfg, A, fp8 ? x_scale : nullptr, rows_cap, expert_offsets, ffn_groups(*cfg), 0,
+                   cfg->H,
                    W1, swiglu ? W3 : nullptr, W2, w.at<void>(w.L.h), y_perm, w.status(), s);
 }
 
@@ -519,7 +538,8 @@ moe_status moe_layer_forward(const moe_config *cfg, const void *x, const void *W
         return MOE_OK;
     }
     const int64_t rows_cap = c.T * c.k;
-    st = run_ffn(c, xg, fp8 ? w.at<float>(w.L.x_scale) : nullptr, rows_cap, offsets, c.N, 0, c.H,
+    st = run_ffn(c, xg, fp8 ? w.at<float>(w.L.x_scale) : nullptr, rows_cap, offsets, ffn_groups(c),
+                 0, c.H,
                  W1, swiglu ? W3 : nullptr, W2, w.at<void>(w.L.h), w.at<void>(w.L.y_perm),
                  w.status(), s, 3);
     if (st != MOE_OK)
