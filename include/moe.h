@@ -219,6 +219,31 @@ moe_status moe_expert_ffn(const moe_config *cfg, const void *x_perm, const float
                           const void *W2, void *y_perm,
                           void *workspace, size_t workspace_bytes, void *stream);
 
+/* Stage 3 for rows that arrive from several ranks ("MoE: what it costs to
+ * train and serve", Expert parallelism and two all-to-alls, step 2: each GPU
+ * runs its local experts on the tokens the first all-to-all brought it).
+ * cfg->N is the number of experts held here; the rows come as n_src blocks,
+ * one per sending rank, each grouped by these N experts.
+ *   x_rows   [rows_cap, d] dispatch_dtype (FP8: E4M3 codes)
+ *   x_scale  [rows_cap] fp32 for FP8 rows, else NULL
+ *   offsets  [n_src*N + 1] int32 (device): the rows of source s for expert e
+ *            are [offsets[s*N + e], offsets[s*N + e + 1]); group (s, e) uses
+ *            weight block e of W1, W3, W2 (laid out as for moe_expert_ffn)
+ *   y_rows   [rows_cap, d] dtype out; rows >= offsets[n_src*N] untouched
+ *   rows_cap rows allocated in x_rows and y_rows, at most cfg->T * cfg->k (the
+ *            workspace holds the hidden activations of that many rows: size
+ *            cfg->T for the rows this rank can receive)
+ * Requires 1 <= n_src and n_src * N <= 1024.  With MOE_OVERFLOW_FALLBACK in
+ * cfg: MOE_ERR_UNSUPPORTED (place the fallback among the N local experts).
+ * The pages have no counterpart to this entry point beyond the step above: it
+ * exists so that the expert-parallel flow can run the local experts on rows
+ * received from every rank in one launch per projection. */
+moe_status moe_expert_ffn_multi(const moe_config *cfg, int32_t n_src, int64_t rows_cap,
+                                const void *x_rows, const float *x_scale,
+                                const int32_t *offsets, const void *W1, const void *W3,
+                                const void *W2, void *y_rows, void *workspace,
+                                size_t workspace_bytes, void *stream);
+
 /* Stage 4, combine ("moe communication costs", Router design, the weighted
  * sum; "MoE: what it costs to train and serve", step 3).
  *   y_perm   [T*k, d] dtype

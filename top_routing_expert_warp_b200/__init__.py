@@ -28,7 +28,7 @@ MOE_OVERFLOW_DROP, MOE_OVERFLOW_FALLBACK = 0, 1
 EXPORTS = ("moe_workspace_bytes", "moe_router", "moe_dispatch", "moe_expert_ffn", "moe_combine",
            "moe_layer_forward", "moe_check_status", "moe_status_string", "moe_last_error_string",
            "moe_version", "moe_launch_count", "moe_profile_begin", "moe_profile_end",
-           "moe_dispatch_noalloc")
+           "moe_dispatch_noalloc", "moe_expert_ffn_multi")
 PROFILE_STAGES = ("router", "dispatch", "expert_up", "expert_down", "shared_expert", "combine")
 
 
@@ -73,12 +73,14 @@ def lib():
         L.moe_dispatch_noalloc.argtypes = [cfgp, P, P, P, P, P, P, P, P, P, P, P, P, P]
         L.moe_dispatch_noalloc.restype = ctypes.c_int
         L.moe_expert_ffn.argtypes = [cfgp, P, P, P, P, P, P, P, P, ctypes.c_size_t, P]
+        L.moe_expert_ffn_multi.argtypes = [cfgp, ctypes.c_int32, ctypes.c_int64, P, P, P, P, P, P, P,
+                                           P, ctypes.c_size_t, P]
         L.moe_combine.argtypes = [cfgp, P, P, P, P, P, P, ctypes.c_size_t, P]
         L.moe_layer_forward.argtypes = [cfgp, P, P, P, P, P, P, P, P, P, P, P, P, P, P, P, P, P,
                                         ctypes.c_size_t, P]
         L.moe_check_status.argtypes = [P, P, ctypes.POINTER(ctypes.c_uint32)]
-        for f in ("moe_router", "moe_dispatch", "moe_expert_ffn", "moe_combine",
-                  "moe_layer_forward", "moe_check_status"):
+        for f in ("moe_router", "moe_dispatch", "moe_expert_ffn", "moe_expert_ffn_multi",
+                  "moe_combine", "moe_layer_forward", "moe_check_status"):
             getattr(L, f).restype = ctypes.c_int
         L.moe_status_string.argtypes = [ctypes.c_int]
         L.moe_status_string.restype = ctypes.c_char_p
@@ -188,6 +190,16 @@ def moe_expert_ffn(cfg, x_perm, x_scale, expert_offsets, W1, W3, W2, y_perm, wor
                                 _ptr(workspace), workspace.numel() * workspace.element_size(),
                                 _stream(stream)),
            "moe_expert_ffn")
+
+
+def moe_expert_ffn_multi(cfg, n_src, rows_cap, x_rows, x_scale, offsets, W1, W3, W2, y_rows,
+                         workspace, stream=None):
+    _check(lib().moe_expert_ffn_multi(ctypes.byref(cfg), int(n_src), int(rows_cap), _ptr(x_rows),
+                                      _ptr(x_scale), _ptr(offsets), _ptr(W1), _ptr(W3), _ptr(W2),
+                                      _ptr(y_rows), _ptr(workspace),
+                                      workspace.numel() * workspace.element_size(),
+                                      _stream(stream)),
+           "moe_expert_ffn_multi")
 
 
 def moe_combine(cfg, y_perm, inv_row, topk_w, y_shared, y, workspace, stream=None):

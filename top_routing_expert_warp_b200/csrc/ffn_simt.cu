@@ -19,8 +19,8 @@ template <int EPI>
 __global__ void __launch_bounds__(kThreads)
     simt_gemm_f32_kernel(const float *__restrict__ A, int64_t rows_cap, int K,
                          const float *__restrict__ B, const float *__restrict__ B2, int n_out,
-                         const int32_t *__restrict__ offsets, int G, int rows_single,
-                         float *__restrict__ out)
+                         const int32_t *__restrict__ offsets, int G, int w_blocks,
+                         int rows_single, float *__restrict__ out)
 {
     grid_dep_wait();
     extern __shared__ float s_a[];
@@ -38,7 +38,7 @@ __global__ void __launch_bounds__(kThreads)
                 else
                     hi = mid;
             }
-            g = lo;
+            g = lo % w_blocks;   // the group's weight block
         }
         __syncthreads();
         for (int i = threadIdx.x; i < K; i += kThreads)
@@ -70,9 +70,11 @@ __global__ void __launch_bounds__(kThreads)
 
 cudaError_t launch_simt_gemm_f32(int epi, const float *A, int64_t rows_cap, int32_t K,
                                  const float *B, const float *B2, int32_t n_out,
-                                 const int32_t *offsets, int32_t G, int32_t rows_single,
-                                 float *out, cudaStream_t stream)
+                                 const int32_t *offsets, int32_t G, int32_t w_blocks,
+                                 int32_t rows_single, float *out, cudaStream_t stream)
 {
+    if (w_blocks <= 0)
+        w_blocks = G;
     if (rows_cap == 0)
         return cudaSuccess;
     int sms = 148, dev = 0;
@@ -84,13 +86,13 @@ cudaError_t launch_simt_gemm_f32(int epi, const float *A, int64_t rows_cap, int3
         return cudaErrorInvalidValue;
     if (epi == EPI_SWIGLU)
         launch_k(simt_gemm_f32_kernel<EPI_SWIGLU>, static_cast<int>(grid), kThreads, smem, stream, 
-            A, rows_cap, K, B, B2, n_out, offsets, G, rows_single, out);
+            A, rows_cap, K, B, B2, n_out, offsets, G, w_blocks, rows_single, out);
     else if (epi == EPI_RELU)
         launch_k(simt_gemm_f32_kernel<EPI_RELU>, static_cast<int>(grid), kThreads, smem, stream, 
-            A, rows_cap, K, B, B2, n_out, offsets, G, rows_single, out);
+            A, rows_cap, K, B, B2, n_out, offsets, G, w_blocks, rows_single, out);
     else
         launch_k(simt_gemm_f32_kernel<EPI_STORE>, static_cast<int>(grid), kThreads, smem, stream, 
-            A, rows_cap, K, B, B2, n_out, offsets, G, rows_single, out);
+            A, rows_cap, K, B, B2, n_out, offsets, G, w_blocks, rows_single, out);
     count_launches(1);
     return cudaGetLastError();
 }

@@ -53,6 +53,7 @@ struct GemmParams {
     const int32_t *offsets;  // [G+1] row offsets of the groups in A, or null
     int32_t rows_single;     // rows of the only group when offsets is null
     int32_t G;
+    int32_t w_blocks;        // group g uses weight block g % w_blocks
     int32_t n_out;           // output columns per group (= rows of B per group)
     int32_t K;
     void *out;
@@ -317,7 +318,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             int pf_t = blockIdx.x, pf_kb = 0, pf_kb1 = 0, pf_brow = 0;
             if (pf_t < total_tiles) {
                 const TileInfo pi = tile_info(pf_t, s_prefix, s_off, G, n_tiles, OUTN, p.ksplit, KB, Geo::REM_ROWS);
-                pf_brow = pi.g * p.n_out + pi.n0;
+                pf_brow = (pi.g % p.w_blocks) * p.n_out + pi.n0;
                 pf_kb = pi.kb0;
                 pf_kb1 = pi.kb1;
             }
@@ -331,7 +332,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                     pf_t += gridDim.x;
                     if (pf_t < total_tiles) {
                         const TileInfo pi = tile_info(pf_t, s_prefix, s_off, G, n_tiles, OUTN, p.ksplit, KB, Geo::REM_ROWS);
-                        pf_brow = pi.g * p.n_out + pi.n0;
+                        pf_brow = (pi.g % p.w_blocks) * p.n_out + pi.n0;
                         pf_kb = pi.kb0;
                         pf_kb1 = pi.kb1;
                     }
@@ -341,7 +342,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                 prefetch_next();
             for (int t = blockIdx.x; t < total_tiles && ok; t += gridDim.x) {
                 const TileInfo ti = tile_info(t, s_prefix, s_off, G, n_tiles, OUTN, p.ksplit, KB, Geo::REM_ROWS);
-                const int brow = ti.g * p.n_out + ti.n0;
+                const int brow = (ti.g % p.w_blocks) * p.n_out + ti.n0;
                 const int a_boxes = ti.ntok / 16;          // swapped tile: 16-row boxes
                 const int r_boxes = ti.rem_ntok / 16;      // combined tile: leftover rows
                 const uint32_t bytes =
@@ -691,6 +692,7 @@ cudaError_t launch_impl(const GemmLaunch &L, cudaStream_t stream)
     p.offsets = L.offsets;
     p.rows_single = L.rows_single;
     p.G = L.G;
+    p.w_blocks = L.w_blocks > 0 ? L.w_blocks : L.G;
     p.n_out = L.n_out;
     p.K = L.K;
     p.out = L.out;

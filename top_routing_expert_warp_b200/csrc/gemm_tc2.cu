@@ -47,6 +47,7 @@ struct PairParams {
     const int32_t *offsets;
     int32_t rows_single;
     int32_t G;
+    int32_t w_blocks;        // group g uses weight block g % w_blocks
     int32_t n_out;
     int32_t K;
     void *out;
@@ -194,7 +195,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             for (int t = pair; t < total_tiles && ok; t += npairs) {
                 const PairTile ti = pair_tile(t, s_prefix, s_off, G, OUTN);
                 const int arow = ti.row0 + static_cast<int>(rank) * HBM;
-                const int brow = ti.g * p.n_out + ti.n0 +
+                const int brow = (ti.g % p.w_blocks) * p.n_out + ti.n0 +
                                  ((EPI == EPI_SWIGLU) ? 0 : static_cast<int>(rank) * 128);
                 for (int kb = 0; kb < KB; ++kb) {
                     if (!mbar_wait_bounded_cluster(&empty[s], ph ^ 1u, s_abort)) {
@@ -436,6 +437,7 @@ cudaError_t launch_pair_impl(const GemmLaunch &L, cudaStream_t stream)
     p.offsets = L.offsets;
     p.rows_single = L.rows_single;
     p.G = L.G;
+    p.w_blocks = L.w_blocks > 0 ? L.w_blocks : L.G;
     p.n_out = L.n_out;
     p.K = L.K;
     p.out = L.out;

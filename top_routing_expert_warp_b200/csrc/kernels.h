@@ -48,6 +48,7 @@ struct GemmLaunch {
     const int32_t *offsets;  // [G+1] device row offsets, or null for one group of rows_single
     int32_t rows_single;
     int32_t G;
+    int32_t w_blocks;        // weight blocks in B: group g uses block g % w_blocks (0: g)
     int32_t n_out;
     void *out;               // [out_rows, ld_out]
     int64_t out_rows;
@@ -83,8 +84,8 @@ constexpr int64_t kPairMinRowsPerGroup = 512;
 // fp32 CUDA-core grouped GEMM (fp32 layers): see ffn_simt.cu.
 cudaError_t launch_simt_gemm_f32(int epi, const float *A, int64_t rows_cap, int32_t K,
                                  const float *B, const float *B2, int32_t n_out,
-                                 const int32_t *offsets, int32_t G, int32_t rows_single,
-                                 float *out, cudaStream_t stream);
+                                 const int32_t *offsets, int32_t G, int32_t w_blocks,
+                                 int32_t rows_single, float *out, cudaStream_t stream);
 
 // Router: see router.cu.
 struct RouterLaunch {

@@ -306,24 +306,27 @@ moe_status run_dispatch(const moe_config &c, const void *x, const int32_t *topk_
 }
 
 // Dense FFN over grouped rows: up (with activation) into h, down into out.
+// Group g of the rows uses weight block g % w_blocks (w_blocks = 0: block g).
 moe_status run_ffn(const moe_config &c, const void *A, const float *row_scale, int64_t rows_cap,
                    const int32_t *offsets, int32_t G, int32_t rows_single, int32_t H,
                    const void *W1, const void *W3, const void *W2, void *h, void *out,
-                   uint32_t *status, cudaStream_t s, int mark_between = -1)
+                   uint32_t *status, cudaStream_t s, int mark_between = -1, int32_t w_blocks = 0)
 {
     if (rows_cap == 0)
         return MOE_OK;
+    const int32_t wb = w_blocks > 0 ? w_blocks : G;
     const int epi = c.act == MOE_ACT_SWIGLU ? moe::EPI_SWIGLU : moe::EPI_RELU;
     if (c.dtype == MOE_F32) {
         MOE_CUDA(moe::launch_simt_gemm_f32(epi, static_cast<const float *>(A), rows_cap, c.d,
                                            static_cast<const float *>(W1),
-                                           static_cast<const float *>(W3), H, offsets, G,
+                                           static_cast<const float *>(W3), H, offsets, G, wb,
                                            rows_single, static_cast<float *>(h), s));
         if (mark_between >= 0)
             prof_mark(mark_between, s);
         MOE_CUDA(moe::launch_simt_gemm_f32(moe::EPI_STORE, static_cast<const float *>(h), rows_cap,
                                            H, static_cast<const float *>(W2), nullptr, c.d,
-                                           offsets, G, rows_single, static_cast<float *>(out), s));
+                                           offsets, G, wb, rows_single, static_cast<float *>(out),
+                                           s));
         return MOE_OK;
     }
     moe::GemmLaunch U{};
@@ -334,10 +337,11 @@ moe_status run_ffn(const moe_config &c, const void *A, const float *row_scale, i
     U.K = c.d;
     U.B = W1;
     U.B2 = W3;
-    U.b_rows = static_cast<int64_t>(G) * H;
+    U.b_rows = static_cast<int64_t>(wb) * H;
     U.offsets = offsets;
     U.rows_single = rows_single;
     U.G = G;
+    U.w_blocks = wb;
     U.n_out = H;
     U.out = h;
     U.out_rows = rows_cap;
@@ -357,10 +361,11 @@ moe_status run_ffn(const moe_config &c, const void *A, const float *row_scale, i
     Dn.K = H;
     Dn.B = W2;
     Dn.B2 = nullptr;
-    Dn.b_rows = static_cast<int64_t>(G) * c.d;
+    Dn.b_rows = static_cast<int64_t>(wb) * c.d;
     Dn.offsets = offsets;
     Dn.rows_single = rows_single;
     Dn.G = G;
+    Dn.w_blocks = wb;
     Dn.n_out = c.d;
     Dn.out = out;
     Dn.out_rows = rows_cap;
@@ -457,6 +462,44 @@ moe_status moe_expert_ffn(const moe_config *cfg, const void *x_perm, const float
     return run_ffn(*cfg, A, fp8 ? x_scale : nullptr, rows_cap, expert_offsets, ffn_groups(*cfg), 0,
                    cfg->H,
                    W1, swiglu ? W3 : nullptr, W2, w.at<void>(w.L.h), y_perm, w.status(), s);
+}
+
+moe_status moe_expert_ffn_multi(const moe_config *cfg, int32_t n_src, int64_t rows_cap,
+                                const void *x_rows, const float *x_scale,
+                                const int32_t *offsets, const void *W1, const void *W3,
+                                const void *W2, void *y_rows, void *workspace,
+                                size_t workspace_bytes, void *stream)
+{
+    if (!config_ok(cfg))
+        return MOE_ERR_INVALID_ARG;
+    if (n_src < 1 || static_cast<int64_t>(n_src) * cfg->N > 1024 || rows_cap < 0 ||
+        rows_cap > cfg->T * cfg->k)
+        return MOE_ERR_INVALID_ARG;
+    if (has_fallback(*cfg))
+        return MOE_ERR_UNSUPPORTED;
+    const bool swiglu = cfg->act == MOE_ACT_SWIGLU;
+    if (rows_cap > 0 && (!x_rows || !offsets || !W1 || !W2 || !y_rows || (swiglu && !W3) ||
+                         !aligned(x_rows, 16) || !aligned(W1, 16) || !aligned(W2, 16) ||
+                         (swiglu && !aligned(W3, 16)) || !aligned(y_rows, 16)))
+        return MOE_ERR_INVALID_ARG;
+    const bool fp8 = cfg->dispatch_dtype == MOE_FP8_E4M3;
+    if (fp8 && rows_cap > 0 && !x_scale)
+        return MOE_ERR_INVALID_ARG;
+    Ws w;
+    moe_status st = check_ws(cfg, workspace, workspace_bytes, &w);
+    if (st != MOE_OK)
+        return st;
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    const int32_t groups = n_src * cfg->N;
+    const void *A = x_rows;
+    if (fp8 && rows_cap > 0) {
+        MOE_CUDA(moe::launch_fp8_to_bf16(static_cast<const uint8_t *>(x_rows), rows_cap, cfg->d,
+                                         offsets, groups, w.at<void>(w.L.x_gemm), s));
+        A = w.at<void>(w.L.x_gemm);
+    }
+    return run_ffn(*cfg, A, fp8 ? x_scale : nullptr, rows_cap, offsets, groups, 0, cfg->H, W1,
+                   swiglu ? W3 : nullptr, W2, w.at<void>(w.L.h), y_rows, w.status(), s, -1,
+                   cfg->N);
 }
 
 moe_status moe_combine(const moe_config *cfg, const void *y_perm, const int32_t *inv_row,
