@@ -94,3 +94,20 @@ def test_expert_parallel_exchange_matches_single_process(world, cf):
     assert np.array_equal(sends, recvs.T)
     if cf > 0:
         assert sum(g[4] for g in got) > 0      # capacity dropped some pairs
+
+
+def test_send_plan_from_expert_offsets():
+    from top_routing_expert_warp_b200 import ep
+    # 6 experts on 3 ranks (2 each); expert e has e + 1 rows, except expert 4 (none)
+    rows = np.array([1, 2, 3, 4, 0, 6])
+    offsets = np.concatenate([[0], np.cumsum(rows)])
+    sc = ep.send_counts_of(offsets, 3)
+    assert sc.tolist() == [[1, 2], [3, 4], [0, 6]]
+    with pytest.raises(ValueError):
+        ep.send_counts_of(offsets, 4)            # 6 experts do not split over 4 ranks
+    # what rank r receives: row r of every source's send counts
+    recv = np.array([[5, 0], [1, 1], [2, 7]])
+    plan = ep.SendPlan(send_counts=sc, recv_counts=recv)
+    assert plan.send_rows == [3, 7, 6] and plan.recv_rows == [5, 2, 9]
+    # received rows: source-major, then by local expert
+    assert plan.recv_offsets().tolist() == [0, 5, 5, 6, 7, 9, 16]
