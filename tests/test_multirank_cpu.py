@@ -66,3 +66,19 @@ def test_reference_arm_on_a_nonzero_rank_exits_without_work(monkeypatch, capsys)
         steps, warmup = 5, 3
     assert bench.run_reference(A, synth.MIXTRAL) == 0
     assert capsys.readouterr().out == ""
+
+
+def test_algorithmic_bytes_count_the_fallback_expert():
+    # the fallback expert's rows and weights enter the roofline like any expert's
+    import numpy as np
+
+    import bench
+    import synth
+    wl = synth.SWITCH_FALLBACK.with_(T=64, N=4, d=32, H=48)
+    kept = np.array([16, 16, 0, 10])
+    plain = bench.algorithmic(wl, kept)
+    fb = bench.algorithmic(wl, np.append(kept, 22))     # 22 pairs over capacity
+    es = 2
+    assert fb["touched"] == plain["touched"] + 1 and fb["R"] == plain["R"] + 22
+    assert fb["bytes"] - plain["bytes"] == 2 * wl.d * wl.H * es     # W1 and W2 (ReLU)
+    assert fb["flops"] - plain["flops"] == 22 * 2.0 * 2 * wl.d * wl.H
