@@ -109,3 +109,28 @@ def test_node_limited_config_validation(lib):
     # the C struct and its ctypes mirror agree on the appended fields
     import ctypes
     assert ctypes.sizeof(moe.moe_config) == 72
+
+
+def test_config_struct_matches_its_ctypes_mirror():
+    # the header's moe_config fields, in order, against the binding's mirror
+    txt = open(os.path.join(ROOT, "include", "moe.h")).read()
+    body = re.search(r"typedef struct moe_config \{(.*?)\} moe_config;", txt, flags=re.S).group(1)
+    body = re.sub(r"/\*.*?\*/", "", body, flags=re.S)
+    decl = re.findall(r"\b(int64_t|int32_t|float)\s+([^;]+);", body)
+    fields = []
+    for ctype, names in decl:
+        for n in names.split(","):
+            fields.append((n.strip(), ctype))
+    ct = {"int64_t": ctypes.c_int64, "int32_t": ctypes.c_int32, "float": ctypes.c_float}
+    mirror = [(n, t) for n, t in moe.moe_config._fields_]
+    assert [n for n, _ in fields] == [n for n, _ in mirror]
+    assert all(ct[c] is t for (_, c), (_, t) in zip(fields, mirror))
+
+
+def test_capacity_variant_config_validation(lib):
+    ok = dict(T=64, d=128, N=8, k=2, H=128, dtype="bf16", capacity_factor=1.0)
+    assert moe.moe_workspace_bytes(moe.make_config(**ok, overflow="fallback", slot_priority=True)) > 0
+    for field, bad in (("overflow", 2), ("slot_priority", 2), ("overflow", -1)):
+        cfg = moe.make_config(**ok)
+        setattr(cfg, field, bad)
+        assert moe.moe_workspace_bytes(cfg) == 0, (field, bad)
