@@ -111,3 +111,13 @@ def test_send_plan_from_expert_offsets():
     assert plan.send_rows == [3, 7, 6] and plan.recv_rows == [5, 2, 9]
     # received rows: source-major, then by local expert
     assert plan.recv_offsets().tolist() == [0, 5, 5, 6, 7, 9, 16]
+
+
+def test_expert_parallel_rejects_fallback_expert():
+    """The exchange covers offsets[0..N]; a fallback expert's rows would be
+    lost, so the layer refuses such a configuration before any launch."""
+    import top_routing_expert_warp_b200 as moe
+    from top_routing_expert_warp_b200 import ep
+    cfg = moe.make_config(64, 64, 8, 2, 128, capacity_factor=1.0, overflow="fallback")
+    with pytest.raises(ValueError, match="fallback"):
+        ep.ep_layer_forward(cfg, None, None, None, None, None, None)

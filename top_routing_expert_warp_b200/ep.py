@@ -108,6 +108,9 @@ def ep_layer_forward(cfg, x, Wg, bias, W1, W3, W2, *, group=None, Ws1=None, Ws3=
     recv_capacity: rows this rank can receive (default T * k * P).
     Returns (y [T, d], topk_idx [T, k], topk_w [T, k]).
     """
+    from . import MOE_OVERFLOW_FALLBACK
+    if cfg.overflow == MOE_OVERFLOW_FALLBACK:
+        raise ValueError("the fallback expert is not supported by the expert-parallel layer")
     import torch.distributed as dist
     P = dist.get_world_size(group)
     T, k, N, d = cfg.T, cfg.k, cfg.N, cfg.d
