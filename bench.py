@@ -5,10 +5,15 @@
 
 One step = one ``moe_layer_forward`` (router -> dispatch -> grouped expert FFN
 -> combine) over one batch of synthetic tokens whose inputs are resident in
-HBM.  The default workload is the Mixtral-shaped layer (T=4096, d=4096, N=8,
-k=2, SwiGLU H=14336, bf16).  For N > 1 (torchrun) every rank runs its own
-replica on its own tokens (weak scaling, no data-path collective); the time is
-the max over ranks and ``value`` counts the tokens of all ranks.
+HBM.  The headline workload is the DeepSeek-V3-shaped layer (T=4096, d=7168,
+N=256 + 1 shared expert, k=8, SwiGLU H=2048, bf16, FP8-E4M3 dispatch), the
+largest configuration; the line also carries, under ``workloads``, the same
+measurement of every other workload (Tiny fp32, Mixtral-, Switch- and
+Grok-1-shaped layers, and the node-limited and fallback-expert variants),
+taken in the same process.  For N > 1 (torchrun) every rank runs its own
+replica of the headline on its own tokens (weak scaling, no data-path
+collective); the time is the max over ranks and ``value`` counts the tokens
+of all ranks.
 
 ``--impl reference`` times the CPU oracle (fp64, the reference arm) on a
 bounded sample of the same workload on this host's cores.
@@ -303,25 +308,60 @@ def config_of(wl):
 
 
 # ----------------------------------------------------------------- our arm
-def run_ours(args, wl):
+L2_BYTES = 126 * 1024 * 1024
+
+
+def near_ties(wl, x_bits, Wg_bits, bias, idx) -> int:
+    """Tokens whose routing may legitimately differ from an exact computation:
+    the k-th and (k+1)-th largest fp64 logits within 1e-3 relative (with
+    node-limited routing also the topk_groups-th and next node scores, and the
+    k-th / next logits among the chosen nodes' experts).  A reported statistic
+    of the run's batch, computed on the host with numpy in fp64."""
+    x = synth.bf16_to_f32(x_bits).astype(np.float64) if x_bits.dtype == np.uint16 else \
+        x_bits.astype(np.float64)
+    W = synth.bf16_to_f32(Wg_bits).astype(np.float64) if Wg_bits.dtype == np.uint16 else \
+        Wg_bits.astype(np.float64)
+    lg = x @ W.T
+    if bias is not None:
+        lg += bias.astype(np.float64)[None, :]
+    T, N = lg.shape
+    k = wl.k
+
+    def gap_tie(v, j):
+        srt = -np.sort(-v, axis=1)
+        a, b = srt[:, j - 1], srt[:, j]
+        fin = np.isfinite(a) & np.isfinite(b)
+        out = np.zeros(len(v), bool)
+        out[fin] = np.abs(a[fin] - b[fin]) <= 1e-3 * np.maximum(np.abs(a[fin]), np.abs(b[fin]))
+        return out
+
+    tie = gap_tie(lg, k) if k < N else np.zeros(T, bool)
+    if wl.n_groups > 1 and 0 < wl.topk_groups < wl.n_groups:
+        S = N // wl.n_groups
+        m = -(-k // wl.topk_groups)
+        p = np.exp(lg - lg.max(axis=1, keepdims=True))
+        p /= p.sum(axis=1, keepdims=True)
+        node = -np.sort(-p.reshape(T, wl.n_groups, S), axis=2)[:, :, :m].sum(2)
+        tie |= gap_tie(node, wl.topk_groups)
+        chosen = np.zeros((T, wl.n_groups), bool)
+        chosen[np.arange(T)[:, None], idx // S] = True
+        masked = np.where(np.repeat(chosen, S, axis=1), lg, -np.inf)
+        tie |= gap_tie(masked, k)
+    return int(tie.sum())
+
+
+def device_inputs(wl, cache: dict) -> dict:
+    """Device tensors of every input of ``wl`` (seeded, generated on the host
+    one expert slice at a time through pinned memory).  Tensors already in
+    ``cache`` under the same seed, name, shape and scale are reused (the
+    node-limited DeepSeek-shaped variant shares the plain layer's weights)."""
     import torch
-    import top_routing_expert_warp_b200 as moe
-
-    rank, local, world = env_rank()
-    torch.cuda.set_device(local)
-    dist = None
-    if world > 1:
-        import datetime
-        import torch.distributed as dist
-        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
-
-    def barrier():
-        if dist is not None:
-            dist.barrier()
-
     dev = {}
-    t_up = time.perf_counter()
     for name, shape, std, dt in synth.tensor_specs(wl):
+        key = (wl.seed, name, tuple(shape), float(std), dt)
+        if key in cache:
+            dev[name] = cache[key]
+            continue
         tdt = torch.float32 if dt == "f32" else torch.bfloat16
         t = torch.empty(shape, dtype=tdt, device="cuda")
         n = int(np.prod(shape))
@@ -333,12 +373,25 @@ def run_ours(args, wl):
             synth.normal(wl.seed, synth.TENSOR_IDS[name], per, std, dt, start=s0,
                          out=pin_np.view(np.uint16) if dt == "bf16" else pin_np)
             flat[s0:s0 + per].copy_(pinned)
-        dev[name] = t
-    gen_s = time.perf_counter() - t_up
-    cfg = moe.make_config(wl.T, wl.d, wl.N, wl.k, wl.H, H_shared=wl.H_shared,
-                          capacity_factor=wl.capacity_factor, gate_mode=wl.gate_mode,
-                          renormalize=wl.renormalize, act=wl.act, dtype=wl.dtype,
-                          dispatch_dtype=wl.dispatch or None, aux_alpha=wl.aux_alpha)
+        torch.cuda.synchronize()
+        cache[key] = dev[name] = t
+    return dev
+
+
+def measure(wl, dev, args, rank, local, world, dist, headline: bool):
+    """Time ``moe_layer_forward`` of workload ``wl`` on resident inputs.
+
+    Returns the per-workload record (and, for the headline, the e2e and launch
+    figures).  Layers whose whole per-step footprint fits in L2 are timed step by
+    step with L2 flushed between steps; the others in one region of K steps."""
+    import torch
+    import top_routing_expert_warp_b200 as moe
+
+    def barrier():
+        if dist is not None:
+            dist.barrier()
+
+    cfg = moe.config_from(wl)
     ws = moe.workspace(cfg)
     tdt = dev["x"].dtype
     # 4 resident token batches (distinct seeds), rotated per step
@@ -369,18 +422,40 @@ def run_ours(args, wl):
     torch.cuda.synchronize()
     st, word = moe.moe_check_status(ws)
     if st != moe.MOE_OK:
-        raise RuntimeError(f"device status after warm-up: {moe.status_string(st)} ({word:#x})")
-    kept_steps = []
+        raise RuntimeError(f"{wl.name}: device status after warm-up: {moe.status_string(st)} "
+                           f"({word:#x})")
+    C = wl.capacity()
+    kept_steps, stats = [], None
     for i in range(4):                       # routing of each rotated batch
         step(i)
         torch.cuda.synchronize()
-        kept = counts.cpu().numpy().astype(np.int64)
-        if wl.capacity_factor > 0:
-            over = int((kept - np.minimum(kept, wl.capacity())).sum())
-            kept = np.minimum(kept, wl.capacity())
+        cnt = counts.cpu().numpy().astype(np.int64)
+        kept = cnt.copy()
+        over = 0
+        if C >= 0:
+            over = int((cnt - np.minimum(cnt, C)).sum())
+            kept = np.minimum(cnt, C)
             if wl.overflow == "fallback":
                 kept = np.append(kept, over)      # the fallback expert's rows
         kept_steps.append(kept)
+        if i == 0:
+            stats = {"near_ties": None, "rows": int(kept.sum()),
+                     "drops": over if wl.overflow != "fallback" else 0,
+                     "rerouted_to_fallback": over if wl.overflow == "fallback" else 0,
+                     "touched_experts": int(np.count_nonzero(kept)),
+                     "L_aux": float(aux.item()), "aux_alpha": wl.aux_alpha}
+            if rank == 0 and not args.no_near_ties:
+                host_x = synth.normal(wl.seed, synth.TENSOR_IDS["x"], wl.T * wl.d, 1.0,
+                                      wl.dtype).reshape(wl.T, wl.d)
+                spec = {s_[0]: s_ for s_ in synth.tensor_specs(wl)}
+                host_wg = synth.normal(wl.seed, synth.TENSOR_IDS["Wg"], wl.N * wl.d,
+                                       spec["Wg"][2], wl.dtype).reshape(wl.N, wl.d)
+                host_b = (synth.normal(wl.seed, synth.TENSOR_IDS["bias"], wl.N, wl.bias_std, "f32")
+                          if wl.bias_std > 0 else None)
+                stats["near_ties"] = near_ties(wl, host_x, host_wg, host_b, idx.cpu().numpy())
+    alg = [algorithmic(wl, k) for k in kept_steps]
+    flush = statistics.mean(a["bytes"] for a in alg) < 2 * L2_BYTES
+    scratch = torch.empty(2 * L2_BYTES, dtype=torch.uint8, device="cuda") if flush else None
 
     # ---- timed region (device events, max over ranks).  Nothing but the
     # layer calls in it: events recorded between the kernels would cut the
@@ -388,21 +463,33 @@ def run_ours(args, wl):
     barrier()
     torch.cuda.synchronize()
     l0 = moe.moe_launch_count()
-    e0 = torch.cuda.Event(enable_timing=True)
-    e1 = torch.cuda.Event(enable_timing=True)
     with Clocks(local) as clk:
-        e0.record(stream)
-        for i in range(args.steps):
-            step(i)
-        e1.record(stream)
-        torch.cuda.synchronize()
+        if not flush:
+            e0 = torch.cuda.Event(enable_timing=True)
+            e1 = torch.cuda.Event(enable_timing=True)
+            e0.record(stream)
+            for i in range(args.steps):
+                step(i)
+            e1.record(stream)
+            torch.cuda.synchronize()
+            ms_local = e0.elapsed_time(e1) / args.steps
+        else:
+            evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+                   for _ in range(args.steps)]
+            for i in range(args.steps):
+                scratch.fill_(i & 0xFF)           # L2 flush, outside the timed events
+                evs[i][0].record(stream)
+                step(i)
+                evs[i][1].record(stream)
+            torch.cuda.synchronize()
+            ms_local = statistics.mean(a.elapsed_time(b) for a, b in evs)
     launches = moe.moe_launch_count() - l0
     barrier()
-    ms_total = max_over_ranks(e0.elapsed_time(e1), dist, "cuda")
-    ms = ms_total / args.steps
+    ms = max_over_ranks(ms_local, dist, "cuda")
     st, word = moe.moe_check_status(ws)
     if st != moe.MOE_OK:
-        raise RuntimeError(f"device status after timing: {moe.status_string(st)} ({word:#x})")
+        raise RuntimeError(f"{wl.name}: device status after timing: {moe.status_string(st)} "
+                           f"({word:#x})")
 
     # ---- kernel-timing pass: the same steps again with the library's stage
     # events (recorded on the launching stream between the stages); gives the
@@ -410,22 +497,78 @@ def run_ours(args, wl):
     barrier()
     torch.cuda.synchronize()
     moe.moe_profile_begin(args.steps)
-    p0 = torch.cuda.Event(enable_timing=True)
-    p1 = torch.cuda.Event(enable_timing=True)
-    p0.record(stream)
     for i in range(args.steps):
+        if flush:
+            scratch.fill_(i & 0xFF)
         step(i)
-    p1.record(stream)
     torch.cuda.synchronize()
     stages, nrec = moe.moe_profile_end()
     barrier()
-    ms_staged = max_over_ranks(p0.elapsed_time(p1), dist, "cuda") / args.steps
 
-    # ---- end to end through the C ABI with host buffers (pinned): every step
-    # copies its tokens in from the host and its output back.  As a serving
-    # loop would, the copies run on two copy streams with double buffers, so
-    # step i+1's input and step i-1's output move while step i computes; the
-    # timed region ends only after the last output has reached the host.
+    e2e = None
+    if headline:
+        e2e = measure_e2e(wl, xs, y, step, args, dist, stream)
+
+    pk, pk_src = peaks()
+    flops = statistics.mean(a["flops"] for a in alg)
+    byts = statistics.mean(a["bytes"] for a in alg)
+    up_flops = statistics.mean(a["up_flops"] for a in alg)
+    up_bytes = statistics.mean(a["up_bytes"] for a in alg)
+    peak_tf_b = pk["bf16_tflops"]
+    peak_tf_s = pk["bf16_tflops_sustained"]
+    peak_bw = pk["hbm_gbs"]
+    up_ms = stages["expert_up"] / max(1, nrec)
+    kname, ksrc = up_kernel(wl)
+    # bound of the dominant kernel: arithmetic intensity vs the ridge point.
+    # It runs inside a step far shorter than a second, so the burst tensor
+    # peak applies; the sustained one is reported beside it
+    ridge = peak_tf_b * 1e12 / (peak_bw * 1e9)
+    if (up_flops / max(up_bytes, 1)) >= ridge:
+        achieved = up_flops / (up_ms * 1e-3) / 1e12
+        roof = {"kernel": f"{kname} (expert up-projection + activation epilogue)",
+                "bound": "tensor", "achieved": achieved, "peak": peak_tf_b, "unit": "TFLOP/s",
+                "frac": achieved / peak_tf_b, "peak_kind": f"bf16_tflops burst ({pk_src})",
+                "frac_of_sustained_peak": achieved / peak_tf_s,
+                "algorithmic_per_launch": up_flops, "launch_ms": up_ms}
+    else:
+        achieved = up_bytes / (up_ms * 1e-3) / 1e9
+        roof = {"kernel": f"{kname} (expert up-projection + activation epilogue)",
+                "bound": "hbm", "achieved": achieved, "peak": peak_bw, "unit": "GB/s",
+                "frac": achieved / peak_bw, "peak_kind": f"hbm_gbs ({pk_src})",
+                "algorithmic_per_launch": up_bytes, "launch_ms": up_ms}
+    roof["traffic"] = traffic_from_profile("grouped_gemm_up", wl_key(wl), ksrc)
+    # the whole layer against its own roofline (slower of the two bounds)
+    t_roof_meas = max(flops / (peak_tf_b * 1e12), byts / (peak_bw * 1e9))
+    t_roof_spec = max(flops / 2.25e15, byts / 8.0e12)
+    layer = {"active_flops": flops, "algorithmic_bytes": byts,
+             "bound": "tensor" if flops / (peak_tf_b * 1e12) >= byts / (peak_bw * 1e9) else "hbm",
+             "roofline_ms_measured_peaks": 1e3 * t_roof_meas,
+             "roofline_ms_spec_peaks": 1e3 * t_roof_spec,
+             "frac_of_roofline_measured": 1e3 * t_roof_meas / ms,
+             "frac_of_roofline_spec": 1e3 * t_roof_spec / ms}
+    rec = {"ms_per_step": ms, "tokens_per_s": weak_value(wl.T, world, ms),
+           "timing": ("per step between CUDA events, L2 flushed (256 MB write) before each step"
+                      if flush else "one region of K steps between CUDA events; inputs larger "
+                                    "than L2 (expert weights streamed from HBM every step, "
+                                    "token batch rotated over 4 resident copies)"),
+           "roofline": roof, "layer_roofline": layer,
+           "stages_ms": {k: v / max(1, nrec) for k, v in stages.items()},
+           "routing": stats, "clocks": clk.summary(), "config": config_of(wl)}
+    if headline:
+        rec["e2e"] = e2e
+        rec["gpu_launches"] = int(launches)
+    del ws, xs, scratch
+    return rec
+
+
+def measure_e2e(wl, xs, y, step, args, dist, stream):
+    """End to end through the C ABI with host buffers (pinned): every step
+    copies its tokens in from the host and its output back.  As a serving loop
+    would, the copies run on two copy streams with double buffers, so step
+    i+1's input and step i-1's output move while step i computes; the timed
+    region ends only after the last output has reached the host."""
+    import torch
+    tdt = xs[0].dtype
     x_host = [xs[i].cpu().pin_memory() for i in range(4)]
     y_host = [torch.empty((wl.T, wl.d), dtype=tdt).pin_memory() for _ in range(2)]
     xin = [torch.empty_like(xs[0]) for _ in range(2)]
@@ -443,7 +586,8 @@ def run_ours(args, wl):
             xin[b].copy_(x_host[i % 4], non_blocking=True)
             in_ready[b].record(h2d)
 
-    barrier()
+    if dist is not None:
+        dist.barrier()
     torch.cuda.synchronize()
     a0 = torch.cuda.Event(enable_timing=True)
     a1 = torch.cuda.Event(enable_timing=True)
@@ -466,70 +610,72 @@ def run_ours(args, wl):
     stream.wait_stream(d2h)
     a1.record(stream)
     torch.cuda.synchronize()
-    barrier()
+    if dist is not None:
+        dist.barrier()
+    world = dist.get_world_size() if dist is not None else 1
     e2e_ms = max_over_ranks(a0.elapsed_time(a1), dist, "cuda") / e_steps
+    return {"value": weak_value(wl.T, world, e2e_ms), "unit": "tokens/s", "ms_per_step": e2e_ms,
+            "copies": "pinned host buffers, double-buffered on two copy streams overlapping the "
+                      "layer",
+            "h2d_bytes_per_step": int(xs[0].numel() * xs[0].element_size()),
+            "d2h_bytes_per_step": int(y.numel() * y.element_size())}
 
-    pk, pk_src = peaks()
+
+def run_ours(args, wl):
+    import torch
+    import top_routing_expert_warp_b200 as moe
+
+    moe.lib()                            # fails loudly when the library is missing
+    rank, local, world = env_rank()
+    torch.cuda.set_device(local)
+    dist = None
+    if world > 1:
+        import datetime
+        import torch.distributed as dist
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
+
+    cache = {}
+    t_up = time.perf_counter()
+    dev = device_inputs(wl, cache)
+    gen_s = time.perf_counter() - t_up
+    head = measure(wl, dev, args, rank, local, world, dist, headline=True)
+
+    # the other workloads, each measured the same way in this process (one
+    # GPU only: under torchrun the scaling run times the headline alone)
+    extra = {}
+    names = [] if (world > 1 or args.workloads == "none") else \
+        [n for n in (args.workloads.split(",") if args.workloads else synth.WORKLOADS)
+         if n != wl_key(wl)]
+    # workloads sharing the headline's tensors first, then free them
+    names.sort(key=lambda n: 0 if synth.WORKLOADS[n].seed == wl.seed else 1)
+    for n in names:
+        w2 = synth.WORKLOADS[n]
+        if w2.seed != wl.seed and cache:
+            dev = None
+            cache.clear()
+            torch.cuda.empty_cache()
+        d2 = device_inputs(w2, cache)
+        extra[n] = measure(w2, d2, args, rank, local, world, dist, headline=False)
+        del d2
+
     out = None
     if rank == 0:
-        alg = [algorithmic(wl, k) for k in kept_steps]
-        flops = statistics.mean(a["flops"] for a in alg)
-        byts = statistics.mean(a["bytes"] for a in alg)
-        up_flops = statistics.mean(a["up_flops"] for a in alg)
-        up_bytes = statistics.mean(a["up_bytes"] for a in alg)
-        peak_tf_s = pk["bf16_tflops_sustained"]
-        peak_tf_b = pk["bf16_tflops"]
-        peak_bw = pk["hbm_gbs"]
-        up_ms = stages["expert_up"] / max(1, nrec)
-        kname, ksrc = up_kernel(wl)
-        # bound of the dominant kernel: arithmetic intensity vs the ridge point
-        ridge = peak_tf_s * 1e12 / (peak_bw * 1e9)
-        tensor_bound = (up_flops / max(up_bytes, 1)) >= ridge
-        if tensor_bound:
-            achieved = up_flops / (up_ms * 1e-3) / 1e12
-            roof = {"kernel": f"{kname} (expert up-projection + SwiGLU/ReLU epilogue)",
-                    "bound": "tensor", "achieved": achieved, "peak": peak_tf_s, "unit": "TFLOP/s",
-                    "frac": achieved / peak_tf_s, "peak_kind": f"bf16_tflops_sustained ({pk_src})",
-                    "frac_of_burst_peak": achieved / peak_tf_b,
-                    "algorithmic_per_launch": up_flops, "launch_ms": up_ms}
-        else:
-            achieved = up_bytes / (up_ms * 1e-3) / 1e9
-            roof = {"kernel": f"{kname} (expert up-projection + SwiGLU/ReLU epilogue)",
-                    "bound": "hbm", "achieved": achieved, "peak": peak_bw, "unit": "GB/s",
-                    "frac": achieved / peak_bw, "peak_kind": f"hbm_gbs ({pk_src})",
-                    "algorithmic_per_launch": up_bytes, "launch_ms": up_ms}
-        roof["traffic"] = traffic_from_profile("grouped_gemm_up", wl_key(wl), ksrc)
-        # the whole layer against its own roofline (slower of the two bounds)
-        t_roof_meas = max(flops / (peak_tf_b * 1e12), byts / (peak_bw * 1e9))
-        t_roof_spec = max(flops / 2.25e15, byts / 8.0e12)
-        layer = {"active_flops": flops, "algorithmic_bytes": byts,
-                 "bound": "tensor" if flops / (peak_tf_b * 1e12) >= byts / (peak_bw * 1e9) else "hbm",
-                 "roofline_ms_measured_peaks": 1e3 * t_roof_meas,
-                 "roofline_ms_spec_peaks": 1e3 * t_roof_spec,
-                 "frac_of_roofline_measured": 1e3 * t_roof_meas / ms,
-                 "frac_of_roofline_spec": 1e3 * t_roof_spec / ms}
         cpu = None
         if world == 1 and not args.no_cpu_baseline:
             rate, n, secs, desc = oracle_sample(wl, args.cpu_budget)
             cpu = {"value": rate, "unit": "tokens/s", "cores": len(os.sched_getaffinity(0)),
                    "kind": "oracle", "sample": desc, "seconds": secs}
-        clocks = clk.summary()
-        out = {"metric": METRIC, "value": weak_value(wl.T, world, ms), "unit": "tokens/s",
-               "n_gpus": world, "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms,
-               "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": wl.dtype,
+        out = {"metric": METRIC, "value": head["tokens_per_s"], "unit": "tokens/s",
+               "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
+               "ms_per_step": head["ms_per_step"], "higher_is_better": True, "scaling": "weak",
+               "vs_baseline": None, "dtype": wl.dtype,
                "data": "synthetic (seeded SplitMix64 + Box-Muller normals; weights N(0, 1/fan_in))",
-               "config": config_of(wl), "roofline": roof, "layer_roofline": layer,
-               "cpu_baseline": cpu,
-               "e2e": {"value": weak_value(wl.T, world, e2e_ms), "unit": "tokens/s",
-                       "ms_per_step": e2e_ms,
-                       "copies": "pinned host buffers, double-buffered on two copy streams "
-                                 "overlapping the layer",
-                       "h2d_bytes_per_step": int(xs[0].numel() * xs[0].element_size()),
-                       "d2h_bytes_per_step": int(y.numel() * y.element_size())},
-               "gpu_launches": int(launches),
-               "stages_ms": {k: v / max(1, nrec) for k, v in stages.items()},
-               "ms_per_step_with_stage_events": ms_staged,
-               "clocks": clocks, "input_gen_s": gen_s}
+               "config": config_of(wl), "roofline": head["roofline"],
+               "layer_roofline": head["layer_roofline"], "cpu_baseline": cpu,
+               "e2e": head["e2e"], "gpu_launches": head["gpu_launches"],
+               "stages_ms": head["stages_ms"], "routing": head["routing"],
+               "clocks": head["clocks"], "timing": head["timing"], "input_gen_s": gen_s,
+               "workloads": {n: {k: v for k, v in r.items()} for n, r in extra.items()}}
     if dist is not None:
         dist.barrier()
         dist.destroy_process_group()
@@ -551,7 +697,14 @@ def main():
     ap.add_argument("--steps", type=int, default=400)
     ap.add_argument("--warmup", type=int, default=10)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
-    ap.add_argument("--workload", choices=list(synth.WORKLOADS), default="mixtral")
+    ap.add_argument("--workload", choices=list(synth.WORKLOADS), default="deepseek",
+                    help="the headline workload (default: the DeepSeek-V3-shaped layer, the "
+                         "largest configuration)")
+    ap.add_argument("--workloads", default="",
+                    help="comma list of further workloads measured in the same run and reported "
+                         "under 'workloads' (default: all others; 'none' for the headline only)")
+    ap.add_argument("--no-near-ties", action="store_true",
+                    help="skip the host fp64 near-tie count")
     ap.add_argument("--cpu-budget", type=float, default=15.0,
                     help="seconds of oracle work for the cpu_baseline sample")
     ap.add_argument("--no-cpu-baseline", action="store_true")

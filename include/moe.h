@@ -133,6 +133,30 @@ typedef struct moe_config {
  * configuration).  Host only, no CUDA calls. */
 size_t moe_workspace_bytes(const moe_config *cfg);
 
+/* Where moe_layer_forward keeps its intermediate dispatch results inside the
+ * workspace, as byte offsets from the workspace start, so that a caller can
+ * read the dispatch of the fused call ("MoE: what it costs to train and
+ * serve", Expert parallelism step 1, as a local permutation) without running
+ * the stages separately.  After a moe_layer_forward on that workspace has
+ * completed on its stream, the regions hold that call's values, laid out as
+ * the outputs of moe_dispatch of the same name; any later call on the
+ * workspace may overwrite them.  topk_idx, topk_w and counts are filled only
+ * when the caller passed NULL for the corresponding output of
+ * moe_layer_forward.  Host only, no CUDA calls; MOE_ERR_INVALID_ARG on an
+ * invalid configuration or a NULL `out`. */
+typedef struct moe_workspace_regions {
+    size_t topk_idx;   /* [T, k] int32 */
+    size_t topk_w;     /* [T, k] fp32 */
+    size_t counts;     /* [N] int32, before capacity */
+    size_t offsets;    /* [N+1] int32 ([N+2] with MOE_OVERFLOW_FALLBACK) */
+    size_t perm;       /* [T*k] int32, rows < R meaningful */
+    size_t inv_row;    /* [T*k] int32, -1 for a dropped pair */
+    size_t drop;       /* [T*k] uint8 */
+    size_t x_scale;    /* [T*k] fp32 per kept row (FP8 dispatch only) */
+    size_t total;      /* = moe_workspace_bytes(cfg) */
+} moe_workspace_regions;
+moe_status moe_workspace_layout(const moe_config *cfg, moe_workspace_regions *out);
+
 /* Stage 1, router ("moe communication costs", Router design; "Advanced GPU
  * Optimization ... Part 5", section 1.1).
  *   x        [T, d]  dtype

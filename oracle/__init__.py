@@ -339,6 +339,43 @@ def forward_rows_lazy(wl, x: np.ndarray, routing: dict, tokens, get_expert, shar
     return layer_rows(wl.act, xin, lidx, gate, drop, W1, W3, W2, **sh)
 
 
+def forward_rows_by_expert(wl, x: np.ndarray, routing: dict, tokens, get_expert,
+                           shared=None) -> np.ndarray:
+    """Layer output y [len(tokens), d] in fp64, the same sum as ``forward_rows``,
+    y_t = sum over kept slots j of g_tj * E_e(t,j)(x_t) (+ shared(x_t))
+    ("moe communication costs", Router design), evaluated expert by expert so
+    that only one expert's weights are held at a time: each expert's pairs go
+    through ``layer_rows`` as one-slot rows with weight 1, then the slots are
+    weighed and summed in slot order, then the shared expert is added.
+    ``get_expert(e)`` returns (W1e [H,d], W3e or None, W2e [d,H])."""
+    tokens = np.asarray(tokens, dtype=np.int64)
+    n, k, d = len(tokens), wl.k, wl.d
+    xr = x[tokens]
+    xin = expert_inputs(wl, xr)
+    idx = _effective_experts(wl, routing)[tokens]
+    gate = routing["gate"][tokens]
+    drop = routing["drop"].reshape(wl.T, wl.k)[tokens]
+    Y = np.zeros((n, k, d))
+    live = drop == 0
+    for e in sorted(set(int(v) for v in idx[live].ravel())):
+        sel = np.argwhere((idx == e) & live)            # (position in tokens, slot)
+        W1e, W3e, W2e = get_expert(e)
+        m = len(sel)
+        Y[sel[:, 0], sel[:, 1]] = layer_rows(
+            wl.act, xin[sel[:, 0]], np.zeros((m, 1), np.int32), np.ones((m, 1)),
+            np.zeros((m, 1), np.uint8), W1e[None], None if W3e is None else W3e[None], W2e[None])
+    y = np.zeros((n, d))
+    for j in range(k):
+        y[live[:, j]] += gate[live[:, j], j, None] * Y[live[:, j], j]
+    if shared is not None:
+        Ws1, Ws3, Ws2 = shared
+        # every routed slot marked dropped: layer_rows then returns the shared expert alone
+        y += layer_rows(wl.act, np.zeros((n, d)), np.zeros((n, 1), np.int32), np.zeros((n, 1)),
+                        np.ones((n, 1), np.uint8), Ws1[None], None if Ws3 is None else Ws3[None],
+                        Ws2[None], xsh=decode(xr), Ws1=Ws1, Ws3=Ws3, Ws2=Ws2)
+    return y
+
+
 def combine(y_rows: np.ndarray, inv_row: np.ndarray, gate: np.ndarray, y_shared=None) -> np.ndarray:
     """y[t] = sum over kept slots j of gate[t,j] * y_rows[inv_row[t*k+j]] (+ y_shared[t]).
 

@@ -14,12 +14,7 @@ import top_routing_expert_warp_b200 as moe
 
 
 def cfg_of(wl: synth.Workload) -> moe.moe_config:
-    return moe.make_config(wl.T, wl.d, wl.N, wl.k, wl.H, H_shared=wl.H_shared,
-                           capacity_factor=wl.capacity_factor, gate_mode=wl.gate_mode,
-                           renormalize=wl.renormalize, act=wl.act, dtype=wl.dtype,
-                           dispatch_dtype=wl.dispatch or None, aux_alpha=wl.aux_alpha,
-                           n_groups=wl.n_groups, topk_groups=wl.topk_groups,
-                           overflow=wl.overflow, slot_priority=wl.slot_priority)
+    return moe.config_from(wl)
 
 
 def tdtype(wl: synth.Workload):

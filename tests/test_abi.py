@@ -134,3 +134,29 @@ def test_capacity_variant_config_validation(lib):
         cfg = moe.make_config(**ok)
         setattr(cfg, field, bad)
         assert moe.moe_workspace_bytes(cfg) == 0, (field, bad)
+
+
+def test_workspace_layout_regions(lib):
+    # host-only: the regions of the layer's intermediates lie inside the workspace,
+    # 256-byte aligned, in the header's order, each large enough for its array
+    cfg = moe.make_config(4096, 7168, 256, 8, 2048, H_shared=2048, gate_mode="F",
+                          renormalize=True, dispatch_dtype="fp8")
+    r = moe.moe_workspace_layout(cfg)
+    assert r["total"] == moe.moe_workspace_bytes(cfg)
+    order = ["topk_idx", "topk_w", "counts", "offsets", "perm", "inv_row", "drop", "x_scale"]
+    offs = [r[n] for n in order]
+    assert all(o % 256 == 0 for o in offs) and offs == sorted(offs) and offs[-1] < r["total"]
+    rows = 4096 * 8
+    need = {"topk_idx": rows * 4, "topk_w": rows * 4, "counts": 256 * 4, "offsets": 258 * 4,
+            "perm": rows * 4, "inv_row": rows * 4, "drop": rows, "x_scale": rows * 4}
+    nxt = offs[1:] + [r["total"]]
+    for n, o, e in zip(order, offs, nxt):
+        assert e - o >= need[n], n
+    # the ctypes mirror has the header's fields in order
+    txt = open(os.path.join(ROOT, "include", "moe.h")).read()
+    body = re.search(r"typedef struct moe_workspace_regions \{(.*?)\} moe_workspace_regions;", txt,
+                     flags=re.S).group(1)
+    body = re.sub(r"/\*.*?\*/", "", body, flags=re.S)
+    assert re.findall(r"size_t\s+(\w+);", body) == [n for n, _ in moe.moe_workspace_regions._fields_]
+    with pytest.raises(moe.MoeError):
+        moe.moe_workspace_layout(moe.make_config(16, 64, 8, 9, 128))   # k > 8

@@ -123,6 +123,31 @@ def test_lazy_rows_equal_stacked_rows():
     assert np.array_equal(a, b)
 
 
+@pytest.mark.parametrize("variant", ["fp8-shared-drop", "fallback-slot"])
+def test_rows_by_expert_equal_stacked_rows(variant):
+    # the expert-by-expert evaluation (one expert's weights at a time) gives the
+    # same sum as the per-token evaluation pinned above against numpy FFNs
+    if variant == "fp8-shared-drop":
+        wl = synth.Workload("byexp", T=40, d=16, N=4, k=2, H=24, act="swiglu", dtype="bf16",
+                            gate_mode="F", renormalize=True, capacity_factor=1.0, H_shared=8,
+                            dispatch="fp8", seed=12)
+    else:
+        wl = synth.Workload("byexp-fb", T=50, d=16, N=4, k=2, H=8, act="relu", dtype="bf16",
+                            gate_mode="R", capacity_factor=0.6, overflow="fallback",
+                            slot_priority=True, seed=14)
+    inp = synth.make_host(wl)
+    routing = oracle.route(wl, inp["x"], inp["Wg"])
+    assert routing["drop"].sum() > 0 or wl.overflow == "fallback"
+    toks = np.arange(wl.T)
+    a = oracle.forward_rows(wl, inp, routing, toks)
+    shared = (inp["Ws1"], inp.get("Ws3"), inp["Ws2"]) if wl.H_shared else None
+    b = oracle.forward_rows_by_expert(
+        wl, inp["x"], routing, toks,
+        lambda e: (inp["W1"][e], inp["W3"][e] if wl.act == "swiglu" else None, inp["W2"][e]),
+        shared)
+    np.testing.assert_allclose(b, a, rtol=1e-13, atol=1e-14)
+
+
 def test_combine_bruteforce():
     T, k, d = 17, 3, 5
     rng_rows = synth.normal(1, 40, 30 * d, 1.0, "f32").reshape(30, d).astype(np.float64)

@@ -28,7 +28,7 @@ MOE_OVERFLOW_DROP, MOE_OVERFLOW_FALLBACK = 0, 1
 EXPORTS = ("moe_workspace_bytes", "moe_router", "moe_dispatch", "moe_expert_ffn", "moe_combine",
            "moe_layer_forward", "moe_check_status", "moe_status_string", "moe_last_error_string",
            "moe_version", "moe_launch_count", "moe_profile_begin", "moe_profile_end",
-           "moe_dispatch_noalloc", "moe_expert_ffn_multi")
+           "moe_dispatch_noalloc", "moe_expert_ffn_multi", "moe_workspace_layout")
 PROFILE_STAGES = ("router", "dispatch", "expert_up", "expert_down", "shared_expert", "combine")
 
 
@@ -42,6 +42,12 @@ class moe_config(ctypes.Structure):
                 ("aux_alpha", ctypes.c_float), ("n_groups", ctypes.c_int32),
                 ("topk_groups", ctypes.c_int32), ("overflow", ctypes.c_int32),
                 ("slot_priority", ctypes.c_int32)]
+
+
+class moe_workspace_regions(ctypes.Structure):
+    """Mirror of ``struct moe_workspace_regions`` in include/moe.h."""
+    _fields_ = [(n, ctypes.c_size_t) for n in ("topk_idx", "topk_w", "counts", "offsets", "perm",
+                                               "inv_row", "drop", "x_scale", "total")]
 
 
 class MoeError(RuntimeError):
@@ -68,6 +74,8 @@ def lib():
         cfgp = ctypes.POINTER(moe_config)
         L.moe_workspace_bytes.argtypes = [cfgp]
         L.moe_workspace_bytes.restype = ctypes.c_size_t
+        L.moe_workspace_layout.argtypes = [cfgp, ctypes.POINTER(moe_workspace_regions)]
+        L.moe_workspace_layout.restype = ctypes.c_int
         L.moe_router.argtypes = [cfgp, P, P, P, P, P, P, P, P, ctypes.c_size_t, P]
         L.moe_dispatch.argtypes = [cfgp, P, P, P, P, P, P, P, P, P, P, P, P, P, ctypes.c_size_t, P]
         L.moe_dispatch_noalloc.argtypes = [cfgp, P, P, P, P, P, P, P, P, P, P, P, P, P]
@@ -150,8 +158,37 @@ def make_config(T, d, N, k, H, *, H_shared=0, capacity_factor=0.0, gate_mode="R"
                       int(bool(slot_priority)))
 
 
+def config_from(spec) -> moe_config:
+    """``make_config`` from any object with the layer's fields as attributes
+    (T, d, N, k, H, act, dtype, gate_mode and, when present, H_shared,
+    capacity_factor, renormalize, dispatch, aux_alpha, n_groups, topk_groups,
+    overflow, slot_priority), so that every switch of the layer is passed."""
+    g = lambda name, default: getattr(spec, name, default)  # noqa: E731
+    return make_config(spec.T, spec.d, spec.N, spec.k, spec.H, H_shared=g("H_shared", 0),
+                       capacity_factor=g("capacity_factor", 0.0), gate_mode=spec.gate_mode,
+                       renormalize=g("renormalize", False), act=spec.act, dtype=spec.dtype,
+                       dispatch_dtype=g("dispatch", None) or None, aux_alpha=g("aux_alpha", 0.01),
+                       n_groups=g("n_groups", 0), topk_groups=g("topk_groups", 0),
+                       overflow=g("overflow", "drop"), slot_priority=g("slot_priority", False))
+
+
 def moe_workspace_bytes(cfg: moe_config) -> int:
     return int(lib().moe_workspace_bytes(ctypes.byref(cfg)))
+
+
+def moe_workspace_layout(cfg: moe_config) -> dict:
+    """Byte offsets of the layer forward's intermediate regions in the workspace."""
+    r = moe_workspace_regions()
+    _check(lib().moe_workspace_layout(ctypes.byref(cfg), ctypes.byref(r)), "moe_workspace_layout")
+    return {n: int(getattr(r, n)) for n, _ in moe_workspace_regions._fields_}
+
+
+def workspace_view(ws, cfg: moe_config, region: str, dtype, count: int):
+    """A typed view of ``count`` elements of a workspace region (no copy)."""
+    import torch
+    off = moe_workspace_layout(cfg)[region]
+    esz = torch.empty((), dtype=dtype).element_size()
+    return ws[off:off + count * esz].view(dtype)
 
 
 def moe_router(cfg, x, Wg, bias, logits, topk_idx, topk_w, p_mean, workspace, stream=None):

@@ -687,16 +687,15 @@ cudaError_t launch_dispatch(const DispatchLaunch &L, cudaStream_t stream)
     int sort_launches;
     if (n_pairs <= kFusedMaxPairs && L.N <= kFusedMaxN) {
         const size_t smem = kFusedWarps * L.N * sizeof(int32_t) + n_pairs * sizeof(int16_t);
-        static bool attr_set = false;   // one size bound for every device and call
-        if (!attr_set) {
-            const cudaError_t err = cudaFuncSetAttribute(
+        static DeviceOnce attr_once;   // per device: function attributes are per device
+        const cudaError_t err = device_once(attr_once, nullptr, [](int *) {
+            return cudaFuncSetAttribute(
                 dispatch_fused_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                 static_cast<int>(kFusedWarps * kFusedMaxN * sizeof(int32_t) +
                                  kFusedMaxPairs * sizeof(int16_t)));
-            if (err != cudaSuccess)
-                return err;
-            attr_set = true;
-        }
+        });
+        if (err != cudaSuccess)
+            return err;
         launch_k(dispatch_fused_kernel, 1, kFusedThreads, smem, stream, L.topk_idx, L.T, L.k,
                  L.slot_priority, L.N, L.capacity, L.fallback, L.counts, L.offsets, L.perm,
                  L.inv_row, L.drop, L.p_mean, L.f, L.aux_loss, L.aux_alpha, L.status);

@@ -650,16 +650,19 @@ bool make_map_bf16(CUtensorMap *m, const void *base, int64_t rows, int64_t cols,
     return r == CUDA_SUCCESS;
 }
 
+// SMs of the current device.
 int sm_count()
 {
-    static int n = 0;
-    if (n == 0) {
-        int dev = 0;
-        cudaGetDevice(&dev);
-        cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev);
-        if (n <= 0)
-            n = 148;
-    }
+    static DeviceOnce once;
+    int n = 0;
+    if (device_once(once, &n, [](int *v) {
+            int dev = 0;
+            cudaError_t e = cudaGetDevice(&dev);
+            if (e == cudaSuccess)
+                e = cudaDeviceGetAttribute(v, cudaDevAttrMultiProcessorCount, dev);
+            return e;
+        }) != cudaSuccess || n <= 0)
+        n = 148;
     return n;
 }
 
@@ -679,15 +682,13 @@ cudaError_t launch_impl(const GemmLaunch &L, cudaStream_t stream)
     } else {
         mB2 = mB;
     }
-    static bool attr_set = false;
-    if (!attr_set) {
-        cudaError_t e = cudaFuncSetAttribute(grouped_gemm_tc<BN, EPI, OUT_F32>,
-                                             cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                             Geo::SMEM_BYTES);
-        if (e != cudaSuccess)
-            return e;
-        attr_set = true;
-    }
+    static DeviceOnce attr_once;   // per device: function attributes are per device
+    cudaError_t e = device_once(attr_once, nullptr, [](int *) {
+        return cudaFuncSetAttribute(grouped_gemm_tc<BN, EPI, OUT_F32>,
+                                    cudaFuncAttributeMaxDynamicSharedMemorySize, Geo::SMEM_BYTES);
+    });
+    if (e != cudaSuccess)
+        return e;
     GemmParams p;
     p.offsets = L.offsets;
     p.rows_single = L.rows_single;

@@ -409,13 +409,14 @@ cudaError_t launch_pair_impl(const GemmLaunch &L, cudaStream_t stream)
     } else {
         mB2 = mB;
     }
-    static int max_pairs = 0;
-    if (max_pairs == 0) {
-        cudaError_t e = cudaFuncSetAttribute(grouped_gemm_tc_pair<EPI>,
-                                             cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                             SMEM_BYTES);
-        if (e != cudaSuccess)
-            return e;
+    static DeviceOnce pair_once;   // per device: function attributes are per device
+    int max_pairs = 0;
+    cudaError_t e = device_once(pair_once, &max_pairs, [](int *v) {
+        cudaError_t err = cudaFuncSetAttribute(grouped_gemm_tc_pair<EPI>,
+                                               cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                               SMEM_BYTES);
+        if (err != cudaSuccess)
+            return err;
         cudaLaunchConfig_t cfg = {};
         cudaLaunchAttribute attr[1];
         attr[0].id = cudaLaunchAttributeClusterDimension;
@@ -428,11 +429,16 @@ cudaError_t launch_pair_impl(const GemmLaunch &L, cudaStream_t stream)
         cfg.attrs = attr;
         cfg.numAttrs = 1;
         int n = 0;
-        e = cudaOccupancyMaxActiveClusters(&n, grouped_gemm_tc_pair<EPI>, &cfg);
-        if (e != cudaSuccess || n <= 0)
-            return e != cudaSuccess ? e : cudaErrorInvalidConfiguration;
-        max_pairs = n;
-    }
+        err = cudaOccupancyMaxActiveClusters(&n, grouped_gemm_tc_pair<EPI>, &cfg);
+        if (err != cudaSuccess)
+            return err;
+        if (n <= 0)
+            return cudaErrorInvalidConfiguration;
+        *v = n;
+        return cudaSuccess;
+    });
+    if (e != cudaSuccess)
+        return e;
     PairParams p;
     p.offsets = L.offsets;
     p.rows_single = L.rows_single;
@@ -467,7 +473,7 @@ cudaError_t launch_pair_impl(const GemmLaunch &L, cudaStream_t stream)
     cfg.stream = stream;
     cfg.attrs = attr;
     cfg.numAttrs = 2;
-    cudaError_t e = cudaLaunchKernelEx(&cfg, grouped_gemm_tc_pair<EPI>, mA, mB, mB2, p);
+    e = cudaLaunchKernelEx(&cfg, grouped_gemm_tc_pair<EPI>, mA, mB, mB2, p);
     count_launches(1);
     return e;
 }

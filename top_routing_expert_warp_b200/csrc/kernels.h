@@ -3,6 +3,7 @@
 #pragma once
 
 #include <cstdint>
+#include <mutex>
 #include <utility>
 #include <cuda_runtime.h>
 
@@ -32,6 +33,40 @@ inline cudaError_t launch_k(void (*kernel)(KArgs...), dim3 grid, dim3 block, siz
 
 // Count of kernel launches made by the library (reported by moe_launch_count).
 void count_launches(int n);
+
+// One-time set-up per device.  CUDA keeps function attributes (the dynamic
+// shared-memory bound) and occupancy for each device separately, so a value
+// cached for the first device a process used is wrong on a second one.
+// device_once runs init(&value) the first time it is reached with a given
+// device current, under a lock, and afterwards returns that device's value.
+constexpr int kMaxDeviceSlots = 64;
+struct DeviceOnce {
+    std::mutex mu;
+    bool done[kMaxDeviceSlots] = {};
+    int value[kMaxDeviceSlots] = {};
+};
+template <typename F>
+inline cudaError_t device_once(DeviceOnce &once, int *value_out, F init)
+{
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess)
+        return e;
+    if (dev < 0 || dev >= kMaxDeviceSlots)
+        return cudaErrorInvalidDevice;
+    std::lock_guard<std::mutex> lk(once.mu);
+    if (!once.done[dev]) {
+        int v = 0;
+        e = init(&v);
+        if (e != cudaSuccess)
+            return e;
+        once.value[dev] = v;
+        once.done[dev] = true;
+    }
+    if (value_out)
+        *value_out = once.value[dev];
+    return cudaSuccess;
+}
 
 enum EpiKind { EPI_STORE = 0, EPI_RELU = 1, EPI_SWIGLU = 2 };
 

@@ -387,6 +387,23 @@ size_t moe_workspace_bytes(const moe_config *cfg)
     return layout_of(*cfg).total;
 }
 
+moe_status moe_workspace_layout(const moe_config *cfg, moe_workspace_regions *out)
+{
+    if (!config_ok(cfg) || !out)
+        return MOE_ERR_INVALID_ARG;
+    const Layout L = layout_of(*cfg);
+    out->topk_idx = L.topk_idx;
+    out->topk_w = L.topk_w;
+    out->counts = L.counts;
+    out->offsets = L.offsets;
+    out->perm = L.perm;
+    out->inv_row = L.inv_row;
+    out->drop = L.drop;
+    out->x_scale = L.x_scale;
+    out->total = L.total;
+    return MOE_OK;
+}
+
 moe_status moe_router(const moe_config *cfg, const void *x, const void *Wg, const float *bias,
                       float *logits, int32_t *topk_idx, float *topk_w, float *p_mean,
                       void *workspace, size_t workspace_bytes, void *stream)
