@@ -113,14 +113,29 @@ def _check_layer(wl, run, host, stride_tokens, get_expert=None, shared=None, ful
     print(f"\n{wl.name}: {ntie} near-tie tokens of {T} ({int(flipped.sum())} routed the other "
           f"way), {len(tokens)} output rows checked, rel-L2 {err:.2e}, max gate err "
           f"{(relw.max() if relw.size else 0):.2e}")
-    # a near-tie is a rare event for these synthetic logits
-    assert ntie <= max(4, T // 50), f"{ntie} near-ties"
+    # near-ties are exempt from the exact index check; with 256 experts the k-th
+    # and (k+1)-th logits are often close (a few % of tokens), but if they were
+    # the norm the exact check above would say little
+    assert ntie <= max(4, T // 10), f"{ntie} near-ties"
     return ntie
 
 
-@pytest.mark.parametrize("name", list(SMALL))
+# fp32 layers beside the tiny one: without a capacity limit the layer runs as
+# one kernel (mode F with a shared SwiGLU expert and slot-ordered rows, node-
+# limited routing); with one, as the separate stages
+SMALL_F32 = {
+    "tiny-f32-shared-swiglu": synth.TINY_F32.with_(T=300, N=16, k=3, act="swiglu", gate_mode="F",
+                                                    renormalize=True, H_shared=64,
+                                                    slot_priority=True, seed=21),
+    "tiny-f32-nodes": synth.TINY_F32.with_(T=200, N=16, k=4, n_groups=4, topk_groups=2, seed=22),
+    "tiny-f32-capacity": synth.TINY_F32.with_(capacity_factor=0.8, seed=23),
+    "tiny-f32-bias-modeF": synth.TINY_F32.with_(T=777, gate_mode="F", bias_std=1.0, k=1, seed=24),
+}
+
+
+@pytest.mark.parametrize("name", list(SMALL) + list(SMALL_F32))
 def test_layer_small_all_tokens(name):
-    wl = SMALL[name]
+    wl = SMALL[name] if name in SMALL else SMALL_F32[name]
     dev, host = upload_inputs(wl)
     run = LayerRun(wl, dev)
     run()
@@ -128,9 +143,9 @@ def test_layer_small_all_tokens(name):
     _check_layer(wl, run, host, np.arange(wl.T), full_check=True)
 
 
-@pytest.mark.parametrize("name", list(SMALL))
+@pytest.mark.parametrize("name", list(SMALL) + ["tiny-f32-shared-swiglu"])
 def test_layer_deterministic(name):
-    wl = SMALL[name]
+    wl = SMALL[name] if name in SMALL else SMALL_F32[name]
     dev, _ = upload_inputs(wl)
     run = LayerRun(wl, dev)
     y1 = run().clone()

@@ -213,9 +213,16 @@ def test_fallback_layer_adds_the_fallback_expert_for_dropped_slots():
 
 
 def test_capacity_uses_the_fp32_capacity_factor():
-    # the layer configuration carries the capacity factor in fp32; 0.7 rounds to
-    # 0.699999988, so with T = 400 and N = 8, C = floor(34.9999994) = 34, not 35
-    assert float(np.float32(0.7)) * 400 / 8 < 35.0
+    # The layer configuration carries the capacity factor in fp32.  0.7 is not a
+    # binary fraction: its nearest fp32 value is 11744051 / 2^24 (the 24-bit
+    # significand 0.7 * 2^24 = 11744051.2 rounded to the nearest integer), i.e.
+    # 0.699999988079071044921875.  So with T = 400 and N = 8,
+    # C = floor(11744051 * 400 / (8 * 2^24)) = floor(34.99999964...) = 34, not 35.
+    from fractions import Fraction
+    cf32 = Fraction(11744051, 1 << 24)
+    assert abs(cf32 - Fraction(7, 10)) < Fraction(1, 1 << 25)      # the nearest fp32 value
+    assert str(float(cf32)) == "0.699999988079071"
+    assert cf32 * 400 / 8 < 35 and int(cf32 * 400 / 8) == 34
     wl = synth.Workload("c", T=400, d=8, N=8, k=1, H=8, act="relu", dtype="f32", gate_mode="R",
                         capacity_factor=0.7)
     assert wl.capacity() == 34

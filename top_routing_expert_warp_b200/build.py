@@ -20,8 +20,8 @@ BUILD = os.path.join(PKG, "_build")
 LIB = os.path.join(PKG, "libmoe_b200.so")
 
 SOURCES = ["moe_abi.cu", "gemm_tc.cu", "router.cu", "dispatch.cu", "combine.cu", "ffn_simt.cu",
-           "dispatch_noalloc.cu", "gemm_tc2.cu"]
-HEADERS = ["common.cuh", "kernels.h"]
+           "dispatch_noalloc.cu", "gemm_tc2.cu", "layer_small.cu"]
+HEADERS = ["common.cuh", "kernels.h", "router_small.cuh"]
 
 NVCC_FLAGS = ["-gencode", "arch=compute_100a,code=sm_100a", "-O3", "-lineinfo", "-std=c++17",
               "-Xcompiler", "-fPIC", "-Xcompiler", "-Wall", "--expt-relaxed-constexpr",

@@ -139,6 +139,136 @@ __global__ void __launch_bounds__(kThreads)
     }
 }
 
+// Wide rows (d of 2048 bf16 or more): one block per token, each thread a
+// few 16-byte chunks of every slot, all of a pass's loads issued before they
+// are used.  Same arithmetic, in the same order, as combine_kernel.
+constexpr int kTokThreads = 256;
+
+template <bool BF16, int KM>
+__global__ void __launch_bounds__(kTokThreads, 3)
+    combine_token_kernel(const uint8_t *__restrict__ y_perm, const int32_t *__restrict__ inv_row,
+                         const float *__restrict__ topk_w, const uint8_t *__restrict__ y_shared,
+                         uint8_t *__restrict__ y, int64_t T, int d, int k, int64_t rows_cap,
+                         uint32_t *status)
+{
+    grid_dep_wait();
+    __shared__ int32_t s_row[KM];
+    __shared__ float s_g[KM];
+    const int esz = BF16 ? 2 : 4;
+    const int chunks = d * esz / 16;
+    constexpr int U = KM >= 8 ? 1 : (KM >= 4 ? 2 : 4);
+    constexpr int V = BF16 ? 8 : 4;
+    for (int64_t t = blockIdx.x; t < T; t += gridDim.x) {
+        __syncthreads();   // the previous token's slots are no longer read
+        if (threadIdx.x < KM) {
+            const int j = threadIdx.x;
+            int32_t row = -1;
+            float g = 0.0f;
+            if (j < k) {
+                row = inv_row[t * k + j];
+                g = topk_w[t * k + j];
+                if (row >= rows_cap || row < -1) {
+                    set_status(status, DEV_BAD_ROW);
+                    row = -1;
+                }
+            }
+            s_row[j] = row;
+            s_g[j] = g;
+        }
+        __syncthreads();
+        int32_t row[KM];
+        float g[KM];
+#pragma unroll
+        for (int j = 0; j < KM; ++j) {
+            row[j] = s_row[j];
+            g[j] = s_g[j];
+        }
+        for (int c0 = threadIdx.x; c0 < chunks; c0 += kTokThreads * U) {
+            uint4 v[KM][U];
+#pragma unroll
+            for (int j = 0; j < KM; ++j) {
+                const uint4 *src = reinterpret_cast<const uint4 *>(
+                    y_perm + static_cast<int64_t>(row[j] > 0 ? row[j] : 0) * d * esz);
+#pragma unroll
+                for (int u = 0; u < U; ++u) {
+                    const int c = c0 + kTokThreads * u;
+                    v[j][u] = (j < k && row[j] >= 0 && c < chunks) ? __ldg(src + c)
+                                                                   : make_uint4(0, 0, 0, 0);
+                }
+            }
+            uint4 sh[U];
+#pragma unroll
+            for (int u = 0; u < U; ++u) {
+                const int c = c0 + kTokThreads * u;
+                sh[u] = (y_shared != nullptr && c < chunks)
+                            ? __ldg(reinterpret_cast<const uint4 *>(
+                                        y_shared + t * static_cast<int64_t>(d) * esz) + c)
+                            : make_uint4(0, 0, 0, 0);
+            }
+            float acc[U][V];
+#pragma unroll
+            for (int u = 0; u < U; ++u)
+#pragma unroll
+                for (int i = 0; i < V; ++i)
+                    acc[u][i] = 0.0f;
+#pragma unroll
+            for (int j = 0; j < KM; ++j) {
+                if (j < k && row[j] >= 0) {
+#pragma unroll
+                    for (int u = 0; u < U; ++u) {
+                        const uint32_t w[4] = {v[j][u].x, v[j][u].y, v[j][u].z, v[j][u].w};
+                        if (BF16) {
+#pragma unroll
+                            for (int i = 0; i < 4; ++i) {
+                                acc[u][2 * i] = fmaf(g[j], __uint_as_float(w[i] << 16), acc[u][2 * i]);
+                                acc[u][2 * i + 1] =
+                                    fmaf(g[j], __uint_as_float(w[i] & 0xFFFF0000u), acc[u][2 * i + 1]);
+                            }
+                        } else {
+#pragma unroll
+                            for (int i = 0; i < 4; ++i)
+                                acc[u][i] = fmaf(g[j], __uint_as_float(w[i]), acc[u][i]);
+                        }
+                    }
+                }
+            }
+#pragma unroll
+            for (int u = 0; u < U; ++u) {
+                const int c = c0 + kTokThreads * u;
+                if (c >= chunks)
+                    continue;
+                if (y_shared != nullptr) {
+                    const uint32_t w[4] = {sh[u].x, sh[u].y, sh[u].z, sh[u].w};
+                    if (BF16) {
+#pragma unroll
+                        for (int i = 0; i < 4; ++i) {
+                            acc[u][2 * i] += __uint_as_float(w[i] << 16);
+                            acc[u][2 * i + 1] += __uint_as_float(w[i] & 0xFFFF0000u);
+                        }
+                    } else {
+#pragma unroll
+                        for (int i = 0; i < 4; ++i)
+                            acc[u][i] += __uint_as_float(w[i]);
+                    }
+                }
+                uint4 o;
+                if (BF16) {
+                    o.x = pack_bf16x2(acc[u][0], acc[u][1]);
+                    o.y = pack_bf16x2(acc[u][2], acc[u][3]);
+                    o.z = pack_bf16x2(acc[u][4], acc[u][5]);
+                    o.w = pack_bf16x2(acc[u][6], acc[u][7]);
+                } else {
+                    o.x = __float_as_uint(acc[u][0]);
+                    o.y = __float_as_uint(acc[u][1]);
+                    o.z = __float_as_uint(acc[u][2]);
+                    o.w = __float_as_uint(acc[u][3]);
+                }
+                reinterpret_cast<uint4 *>(y + t * static_cast<int64_t>(d) * esz)[c] = o;
+            }
+        }
+    }
+}
+
 }  // namespace
 
 cudaError_t launch_combine(int dtype, const void *y_perm, const int32_t *inv_row,
@@ -158,6 +288,21 @@ cudaError_t launch_combine(int dtype, const void *y_perm, const int32_t *inv_row
     const uint8_t *ys = static_cast<const uint8_t *>(y_shared);
     uint8_t *yo = static_cast<uint8_t *>(y);
     const int g = static_cast<int>(grid);
+    if (dtype == MOE_BF16 && d >= 2048 && k >= 4) {
+        // wide rows and many slots: a block per token
+        const int gt = static_cast<int>(T < static_cast<int64_t>(sms) * 8 ? T : sms * 8);
+        if (k <= 2)
+            launch_k(combine_token_kernel<true, 2>, gt, kTokThreads, 0, stream, yp, inv_row,
+                     topk_w, ys, yo, T, d, k, rows_cap, status);
+        else if (k <= 4)
+            launch_k(combine_token_kernel<true, 4>, gt, kTokThreads, 0, stream, yp, inv_row,
+                     topk_w, ys, yo, T, d, k, rows_cap, status);
+        else
+            launch_k(combine_token_kernel<true, kMaxK>, gt, kTokThreads, 0, stream, yp, inv_row,
+                     topk_w, ys, yo, T, d, k, rows_cap, status);
+        count_launches(1);
+        return cudaGetLastError();
+    }
     if (dtype == MOE_BF16) {
         if (k <= 1)
             launch_k(combine_kernel<true, 1>, g, kThreads, 0, stream, yp, inv_row, topk_w, ys, yo,

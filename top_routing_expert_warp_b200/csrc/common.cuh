@@ -118,6 +118,33 @@ __device__ __forceinline__ void tma_prefetch_desc(const CUtensorMap *m)
     asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(m)) : "memory");
 }
 
+// L2 eviction-priority policies for the cache hints below.
+__device__ __forceinline__ uint64_t l2_policy_evict_first()
+{
+    uint64_t pol;
+    asm volatile("createpolicy.fractional.L2::evict_first.b64 %0, 1.0;" : "=l"(pol));
+    return pol;
+}
+
+__device__ __forceinline__ uint64_t l2_policy_evict_last()
+{
+    uint64_t pol;
+    asm volatile("createpolicy.fractional.L2::evict_last.b64 %0, 1.0;" : "=l"(pol));
+    return pol;
+}
+
+// tma_load_2d with an L2 cache-eviction hint.
+__device__ __forceinline__ void tma_load_2d_hint(void *smem_dst, const CUtensorMap *m,
+                                                 uint64_t *bar, int32_t c0, int32_t c1,
+                                                 uint64_t policy)
+{
+    asm volatile(
+        "cp.async.bulk.tensor.2d.shared::cluster.global.mbarrier::complete_tx::bytes.L2::cache_hint"
+        " [%0], [%1, {%3, %4}], [%2], %5;" ::"r"(smem_u32(smem_dst)),
+        "l"(reinterpret_cast<uint64_t>(m)), "r"(smem_u32(bar)), "r"(c0), "r"(c1), "l"(policy)
+        : "memory");
+}
+
 // 2-D tiled bulk tensor copy global -> shared, completion counted on `bar`
 // in bytes.  c0 is the innermost (contiguous) coordinate in elements.
 __device__ __forceinline__ void tma_load_2d(void *smem_dst, const CUtensorMap *m, uint64_t *bar,
@@ -386,6 +413,33 @@ __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi)
 __device__ __forceinline__ float bf16_bits_to_f32(uint32_t bits16)
 {
     return __uint_as_float(bits16 << 16);
+}
+
+// ------------------------------------------------------------------ cp.async
+// 16-byte copy global -> shared; src_bytes = 0 reads nothing and fills zeros.
+__device__ __forceinline__ void cp_async_16(uint32_t smem_dst, const void *src, uint32_t src_bytes)
+{
+    asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(smem_dst), "l"(src),
+                 "r"(src_bytes)
+                 : "memory");
+}
+
+// cp.async groups of this thread: close the current group; wait until at most
+// N groups are still in flight; wait for all of them.
+__device__ __forceinline__ void cp_async_commit()
+{
+    asm volatile("cp.async.commit_group;" ::: "memory");
+}
+
+template <int N>
+__device__ __forceinline__ void cp_async_wait()
+{
+    asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory");
+}
+
+__device__ __forceinline__ void cp_async_wait_all()
+{
+    asm volatile("cp.async.wait_all;" ::: "memory");
 }
 
 __device__ __forceinline__ uint32_t lanemask_lt()

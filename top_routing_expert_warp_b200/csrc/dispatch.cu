@@ -56,15 +56,20 @@ __global__ void __launch_bounds__(kThreads)
     const int lane = threadIdx.x & 31;
     const int64_t n_pairs = T * k;
     const int64_t base = static_cast<int64_t>(blockIdx.x) * kDispChunk;
-    for (int r = 0; r < kDispChunk / kThreads; ++r) {
+    constexpr int R = kDispChunk / kThreads;
+    int ev[R];   // every load of the thread issued before the first is used
+#pragma unroll
+    for (int r = 0; r < R; ++r) {
         const int64_t p = base + r * kThreads + threadIdx.x;
-        int e = -1;
-        if (p < n_pairs) {
-            e = idx[pair_at(p, T, k, slot_priority)];
-            if (e < 0 || e >= N) {
-                set_status(status, DEV_BAD_EXPERT);
-                e = -1;
-            }
+        ev[r] = p < n_pairs ? idx[pair_at(p, T, k, slot_priority)] : -1;
+    }
+#pragma unroll
+    for (int r = 0; r < R; ++r) {
+        const int64_t p = base + r * kThreads + threadIdx.x;
+        int e = ev[r];
+        if (p < n_pairs && (e < 0 || e >= N)) {
+            set_status(status, DEV_BAD_EXPERT);
+            e = -1;
         }
         const uint32_t peers = __match_any_sync(0xffffffffu, e);
         if (e >= 0 && lane == __ffs(peers) - 1)
@@ -224,18 +229,28 @@ __global__ void __launch_bounds__(1024)
     __syncthreads();
     int32_t run = 0;
     if (e < N) {
-        for (int b = 0; b < nblk; ++b) {
-            const int64_t o = static_cast<int64_t>(b) * N + e;
-            const int32_t v = block_base[o];
-            block_base[o] = run;
-            if (fb) {
-                // pairs of this block past the first C of the expert
-                int64_t over = static_cast<int64_t>(run) + v - C;
-                over = over < 0 ? 0 : (over > v ? v : over);
-                if (over > 0)
-                    atomicAdd(&fb_base[b], static_cast<int32_t>(over));
+        constexpr int B = 8;   // the counts of B blocks loaded together
+        for (int b0 = 0; b0 < nblk; b0 += B) {
+            int32_t vb[B];
+#pragma unroll
+            for (int u = 0; u < B; ++u)
+                vb[u] = b0 + u < nblk ? block_base[static_cast<int64_t>(b0 + u) * N + e] : 0;
+#pragma unroll
+            for (int u = 0; u < B; ++u) {
+                const int b = b0 + u;
+                if (b >= nblk)
+                    break;
+                const int32_t v = vb[u];
+                block_base[static_cast<int64_t>(b) * N + e] = run;
+                if (fb) {
+                    // pairs of this block past the first C of the expert
+                    int64_t over = static_cast<int64_t>(run) + v - C;
+                    over = over < 0 ? 0 : (over > v ? v : over);
+                    if (over > 0)
+                        atomicAdd(&fb_base[b], static_cast<int32_t>(over));
+                }
+                run += v;
             }
-            run += v;
         }
     }
     __syncthreads();
@@ -402,15 +417,19 @@ __global__ void __launch_bounds__(kThreads)
     __syncthreads();
     const int64_t wbase = static_cast<int64_t>(blockIdx.x) * kDispChunk + warp * kPerWarp;
     int32_t *mine = s_w + warp * N;
-    // phase 1: per-warp counts
-    for (int r = 0; r < kPerWarp / 32; ++r) {
+    // this lane's experts of the warp's rounds, loaded once for both walks
+    constexpr int R = kPerWarp / 32;
+    int ev[R];
+#pragma unroll
+    for (int r = 0; r < R; ++r) {
         const int64_t p = wbase + r * 32 + lane;
-        int e = -1;
-        if (p < n_pairs) {
-            e = idx[pair_at(p, T, k, slot_priority)];
-            if (e < 0 || e >= N)
-                e = -1;
-        }
+        int e = p < n_pairs ? idx[pair_at(p, T, k, slot_priority)] : -1;
+        ev[r] = (e < 0 || e >= N) ? -1 : e;
+    }
+    // phase 1: per-warp counts
+#pragma unroll
+    for (int r = 0; r < R; ++r) {
+        const int e = ev[r];
         const uint32_t peers = __match_any_sync(0xffffffffu, e);
         if (e >= 0 && lane == __ffs(peers) - 1)
             mine[e] += __popc(peers);
@@ -429,14 +448,10 @@ __global__ void __launch_bounds__(kThreads)
     __syncthreads();
     // phase 3: walk the pairs in order; rank = warp base + earlier lanes
     int32_t n_over = 0;
-    for (int r = 0; r < kPerWarp / 32; ++r) {
+#pragma unroll
+    for (int r = 0; r < R; ++r) {
         const int64_t p = wbase + r * 32 + lane;
-        int e = -1;
-        if (p < n_pairs) {
-            e = idx[pair_at(p, T, k, slot_priority)];
-            if (e < 0 || e >= N)
-                e = -1;
-        }
+        const int e = ev[r];
         const uint32_t peers = __match_any_sync(0xffffffffu, e);
         int32_t rank = 0;
         if (e >= 0)

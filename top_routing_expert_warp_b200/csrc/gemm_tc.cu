@@ -60,10 +60,25 @@ struct GemmParams {
     int64_t ld_out;          // elements
     const float *row_scale;  // multiply each accumulator row by row_scale[r], or null
     int64_t rows_cap;        // rows allocated in out (and row_scale); rows beyond are never written
-    int32_t prefetch;        // 1: prefetch weight boxes into L2 ahead of their loads
     int32_t ksplit;          // >1: split K; split s writes its partial sums at out + s*split_stride
     int64_t split_stride;    // elements
     uint32_t *status;
+    // Optional second problem (x_rows > 0): one group of x_rows rows with its
+    // own A (tensor maps tmXA, tmXA16), weights (tmXB, tmXB2), reduction
+    // length x_K and output x_out [x_rows, x_ld_out] (n_out columns = x_n_out),
+    // no row scale and no K split.  Its tiles are spread evenly through the
+    // grouped problem's tiles, so that a compute-bound problem (a layer's
+    // always-on shared expert) runs on the tensor cores while the grouped
+    // problem streams its weights from HBM.
+    int32_t x_rows;
+    int32_t x_K;
+    int32_t x_n_out;
+    void *x_out;
+    int64_t x_ld_out;
+    // 1: the grouped problem's weights are streamed once (few rows per group):
+    // load the weight tiles of groups of one or two m tiles evict-first from
+    // L2, and the rows evict-last, since every n tile of a group reads them
+    int32_t stream_hint;
 };
 
 // Leftover rows a combined tile takes (multiple of 16; 256-column tiles only).
@@ -91,10 +106,6 @@ struct Geometry {
 // of 16, its N, so the tensor cores do not pad the rows to 128.
 constexpr int kSwapMaxRows = 112;
 
-// Weight boxes may be prefetched into L2 this many k-blocks before their load
-// (GemmParams::prefetch; helps weight streaming when few CTAs share a tile).
-constexpr int kPrefetchAhead = 8;
-
 struct TileInfo {
     int32_t g, row0, rows_valid, n0;
     bool swap;
@@ -102,6 +113,8 @@ struct TileInfo {
     int32_t ks, kb0, kb1;   // K split index and its k-block range
     bool combo;             // combined tile: rows_valid = 128 plus rem_rows more
     int32_t rem_rows, rem_ntok;
+    bool extra;             // a tile of the second problem
+    int32_t mtiles;         // m tiles of the tile's group
 };
 
 // m tiles of a group of `rows` rows when up to rem_max leftover rows ride
@@ -117,33 +130,22 @@ __host__ __device__ __forceinline__ int m_tiles_of(int rows, int rem_max)
     return (rem == 0 || rem <= rem_max) ? q : q + 1;
 }
 
-// Locate tile t: prefix[g] <= t < prefix[g+1].  Inside a group the order is
-// (K split, n tile, m tile) with m fastest, so CTAs running side by side share
-// the weight tile through L2.
-__device__ __forceinline__ TileInfo tile_info(int t, const int32_t *s_prefix,
-                                              const int32_t *s_off, int G, int n_tiles,
-                                              int outn, int ksplit, int KB, int rem_max)
+// Tile `local` of one group of `rows_g` rows starting at row `row_base`, in
+// the order (K split, n tile, m tile) with m fastest, so CTAs running side by
+// side share the weight tile through L2.
+__device__ __forceinline__ TileInfo group_tile(int g, int local, int row_base, int rows_g,
+                                               int n_tiles, int outn, int ksplit, int KB,
+                                               int rem_max)
 {
-    int lo = 0, hi = G;  // find largest g with prefix[g] <= t
-    while (hi - lo > 1) {
-        int mid = (lo + hi) >> 1;
-        if (s_prefix[mid] <= t)
-            lo = mid;
-        else
-            hi = mid;
-    }
-    int g = lo;
-    int rows_g = s_off[g + 1] - s_off[g];
-    int mt_g = m_tiles_of(rows_g, rem_max);
-    int local = t - s_prefix[g];
+    const int mt_g = m_tiles_of(rows_g, rem_max);
     const int per_split = mt_g * n_tiles;
     const int ks = local / per_split;
     local -= ks * per_split;
-    int n_tile = local / mt_g;
-    int m_tile = local - n_tile * mt_g;
+    const int n_tile = local / mt_g;
+    const int m_tile = local - n_tile * mt_g;
     TileInfo ti;
     ti.g = g;
-    ti.row0 = s_off[g] + m_tile * BM;
+    ti.row0 = row_base + m_tile * BM;
     ti.rows_valid = min(BM, rows_g - m_tile * BM);
     ti.n0 = n_tile * outn;
     const int rest = rows_g - (m_tile + 1) * BM;   // rows past this tile (last tile: <= rem_max)
@@ -155,7 +157,48 @@ __device__ __forceinline__ TileInfo tile_info(int t, const int32_t *s_prefix,
     ti.ks = ks;
     ti.kb0 = static_cast<int>((static_cast<int64_t>(ks) * KB) / ksplit);
     ti.kb1 = static_cast<int>((static_cast<int64_t>(ks + 1) * KB) / ksplit);
+    ti.extra = false;
+    ti.mtiles = mt_g;
     return ti;
+}
+
+// The merged tile list: `routed` tiles of the grouped problem and `extra`
+// tiles of the second problem, the latter at positions t where
+// floor((t + 1) E / total) > floor(t E / total), i.e. evenly spread.
+struct Sched {
+    int routed, extra, total;
+    int x_ntiles, x_KB;
+};
+
+// Locate tile t of the merged list.  Grouped tiles: prefix[g] <= local <
+// prefix[g+1] finds the group.
+__device__ __forceinline__ TileInfo tile_info(int t, const Sched &sc, const int32_t *s_prefix,
+                                              const int32_t *s_off, int G, int n_tiles,
+                                              int outn, int ksplit, int KB, int rem_max,
+                                              int x_rows)
+{
+    int local = t;
+    if (sc.extra > 0) {
+        const int c0 = static_cast<int>((static_cast<int64_t>(t) * sc.extra) / sc.total);
+        const int c1 = static_cast<int>((static_cast<int64_t>(t + 1) * sc.extra) / sc.total);
+        if (c1 > c0) {
+            TileInfo ti = group_tile(0, c0, 0, x_rows, sc.x_ntiles, outn, 1, sc.x_KB, rem_max);
+            ti.extra = true;
+            return ti;
+        }
+        local = t - c0;
+    }
+    int lo = 0, hi = G;  // find largest g with prefix[g] <= local
+    while (hi - lo > 1) {
+        int mid = (lo + hi) >> 1;
+        if (s_prefix[mid] <= local)
+            lo = mid;
+        else
+            hi = mid;
+    }
+    const int g = lo;
+    return group_tile(g, local - s_prefix[g], s_off[g], s_off[g + 1] - s_off[g], n_tiles, outn,
+                      ksplit, KB, rem_max);
 }
 
 __device__ __forceinline__ float silu_f(float a)
@@ -214,7 +257,10 @@ template <int BN, int EPI, bool OUT_F32>
 __global__ void __launch_bounds__(kThreads, 1)
     grouped_gemm_tc(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmA16,
                     const __grid_constant__ CUtensorMap tmB, const __grid_constant__ CUtensorMap tmB2,
-                    GemmParams p)
+                    const __grid_constant__ CUtensorMap tmXA,
+                    const __grid_constant__ CUtensorMap tmXA16,
+                    const __grid_constant__ CUtensorMap tmXB,
+                    const __grid_constant__ CUtensorMap tmXB2, GemmParams p)
 {
     grid_dep_wait();
     using Geo = Geometry<BN, EPI>;
@@ -261,6 +307,13 @@ __global__ void __launch_bounds__(kThreads, 1)
         tma_prefetch_desc(&tmB);
         if (EPI == EPI_SWIGLU)
             tma_prefetch_desc(&tmB2);
+        if (p.x_rows > 0) {
+            tma_prefetch_desc(&tmXA);
+            tma_prefetch_desc(&tmXA16);
+            tma_prefetch_desc(&tmXB);
+            if (EPI == EPI_SWIGLU)
+                tma_prefetch_desc(&tmXB2);
+        }
     }
     if (warp == 1) {
         tmem_alloc(s_tmem, Geo::TMEM_COLS);
@@ -303,7 +356,17 @@ __global__ void __launch_bounds__(kThreads, 1)
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem_base = *s_tmem;
-    const int total_tiles = s_prefix[G];
+    Sched sched;
+    sched.routed = s_prefix[G];
+    sched.x_ntiles = p.x_rows > 0 ? (p.x_n_out + OUTN - 1) / OUTN : 0;
+    sched.extra = p.x_rows > 0 ? m_tiles_of(p.x_rows, Geo::REM_ROWS) * sched.x_ntiles : 0;
+    sched.total = sched.routed + sched.extra;
+    sched.x_KB = (p.x_K + BK - 1) / BK;
+    const int total_tiles = sched.total;
+    auto info = [&](int t) {
+        return tile_info(t, sched, s_prefix, s_off, G, n_tiles, OUTN, p.ksplit, KB, Geo::REM_ROWS,
+                         p.x_rows);
+    };
 
     if (warp == 0) {
         // ================= TMA producer =================
@@ -313,41 +376,35 @@ __global__ void __launch_bounds__(kThreads, 1)
             uint32_t last_par = 0;  // bit s: parity of the last load issued to stage s
             uint32_t used = 0;
             bool ok = true;
-            // L2 prefetch cursor: kPrefetchAhead k-blocks ahead of the loads in
-            // this CTA's own (tile, k-block) sequence, weights only
-            int pf_t = blockIdx.x, pf_kb = 0, pf_kb1 = 0, pf_brow = 0;
-            if (pf_t < total_tiles) {
-                const TileInfo pi = tile_info(pf_t, s_prefix, s_off, G, n_tiles, OUTN, p.ksplit, KB, Geo::REM_ROWS);
-                pf_brow = (pi.g % p.w_blocks) * p.n_out + pi.n0;
-                pf_kb = pi.kb0;
-                pf_kb1 = pi.kb1;
-            }
-            auto prefetch_next = [&]() {
-                if (!p.prefetch || pf_t >= total_tiles)
-                    return;
-                tma_prefetch_l2_2d(&tmB, pf_kb * BK, pf_brow);
-                if (EPI == EPI_SWIGLU)
-                    tma_prefetch_l2_2d(&tmB2, pf_kb * BK, pf_brow);
-                if (++pf_kb >= pf_kb1) {
-                    pf_t += gridDim.x;
-                    if (pf_t < total_tiles) {
-                        const TileInfo pi = tile_info(pf_t, s_prefix, s_off, G, n_tiles, OUTN, p.ksplit, KB, Geo::REM_ROWS);
-                        pf_brow = (pi.g % p.w_blocks) * p.n_out + pi.n0;
-                        pf_kb = pi.kb0;
-                        pf_kb1 = pi.kb1;
-                    }
-                }
-            };
-            for (int i = 0; i < kPrefetchAhead; ++i)
-                prefetch_next();
+            const uint64_t pol_first = l2_policy_evict_first();
+            const uint64_t pol_last = l2_policy_evict_last();
             for (int t = blockIdx.x; t < total_tiles && ok; t += gridDim.x) {
-                const TileInfo ti = tile_info(t, s_prefix, s_off, G, n_tiles, OUTN, p.ksplit, KB, Geo::REM_ROWS);
-                const int brow = (ti.g % p.w_blocks) * p.n_out + ti.n0;
+                const TileInfo ti = info(t);
+                // weights of groups of one or two m tiles are read once or twice in a row
+                const bool hint = p.stream_hint != 0 && !ti.extra && ti.mtiles <= 2;
+                const uint64_t pol_a = hint ? pol_last : 0;
+                const CUtensorMap *mA = ti.extra ? &tmXA : &tmA;
+                const CUtensorMap *mA16 = ti.extra ? &tmXA16 : &tmA16;
+                const CUtensorMap *mB = ti.extra ? &tmXB : &tmB;
+                const CUtensorMap *mB2 = ti.extra ? &tmXB2 : &tmB2;
+                const int brow = ti.extra ? ti.n0 : (ti.g % p.w_blocks) * p.n_out + ti.n0;
                 const int a_boxes = ti.ntok / 16;          // swapped tile: 16-row boxes
                 const int r_boxes = ti.rem_ntok / 16;      // combined tile: leftover rows
                 const uint32_t bytes =
                     ti.swap ? (a_boxes * 16 * BK * 2 + Geo::B_STAGE_BYTES)
                             : (Geo::AB_BYTES + r_boxes * 16 * BK * 2);
+                auto load_a = [&](uint8_t *dst, const CUtensorMap *m, int c0, int c1) {
+                    if (hint)
+                        tma_load_2d_hint(dst, m, &full[s], c0, c1, pol_a);
+                    else
+                        tma_load_2d(dst, m, &full[s], c0, c1);
+                };
+                auto load_b = [&](uint8_t *dst, const CUtensorMap *m, int c0, int c1) {
+                    if (hint)
+                        tma_load_2d_hint(dst, m, &full[s], c0, c1, pol_first);
+                    else
+                        tma_load_2d(dst, m, &full[s], c0, c1);
+                };
                 for (int kb = ti.kb0; kb < ti.kb1; ++kb) {
                     if (!mbar_wait_bounded(&empty[s], ph ^ 1u, s_abort)) {
                         set_status(p.status, DEV_TIMEOUT_PRODUCER);
@@ -360,21 +417,16 @@ __global__ void __launch_bounds__(kThreads, 1)
                     mbar_arrive_expect_tx(&full[s], bytes);
                     if (ti.swap) {
                         for (int b = 0; b < a_boxes; ++b)
-                            tma_load_2d(sa + b * 16 * BK * 2, &tmA16, &full[s], kb * BK,
-                                        ti.row0 + 16 * b);
+                            load_a(sa + b * 16 * BK * 2, mA16, kb * BK, ti.row0 + 16 * b);
                     } else {
-                        tma_load_2d(sa, &tmA, &full[s], kb * BK, ti.row0);
+                        load_a(sa, mA, kb * BK, ti.row0);
                         for (int b = 0; b < r_boxes; ++b)   // leftover rows after the B block
-                            tma_load_2d(sb + Geo::B_STAGE_BYTES + b * 16 * BK * 2, &tmA16,
-                                        &full[s], kb * BK, ti.row0 + BM + 16 * b);
+                            load_a(sb + Geo::B_STAGE_BYTES + b * 16 * BK * 2, mA16, kb * BK,
+                                   ti.row0 + BM + 16 * b);
                     }
-                    if (EPI == EPI_SWIGLU) {
-                        tma_load_2d(sb, &tmB, &full[s], kb * BK, brow);
-                        tma_load_2d(sb + (BN / 2) * BK * 2, &tmB2, &full[s], kb * BK, brow);
-                    } else {
-                        tma_load_2d(sb, &tmB, &full[s], kb * BK, brow);
-                    }
-                    prefetch_next();
+                    load_b(sb, mB, kb * BK, brow);
+                    if (EPI == EPI_SWIGLU)
+                        load_b(sb + (BN / 2) * BK * 2, mB2, kb * BK, brow);
                     last_par = (last_par & ~(1u << s)) | (ph << s);
                     used |= 1u << s;
                     if (++s == STAGES) {
@@ -401,7 +453,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             int it = 0;
             bool ok = true;
             for (int t = blockIdx.x; t < total_tiles && ok; t += gridDim.x) {
-                const TileInfo ti = tile_info(t, s_prefix, s_off, G, n_tiles, OUTN, p.ksplit, KB, Geo::REM_ROWS);
+                const TileInfo ti = info(t);
                 const uint32_t idesc_s = idesc_bf16_f32(128, ti.ntok);
                 const uint32_t idesc_r = idesc_bf16_f32(128, ti.rem_ntok > 0 ? ti.rem_ntok : 16);
                 // accumulator(s): a combined tile takes the next two
@@ -490,13 +542,20 @@ __global__ void __launch_bounds__(kThreads, 1)
             }
             tc_fence_after();
             const uint32_t tacc = tmem_base + (static_cast<uint32_t>(q * 32) << 16) + a * BN;
+            // output of the tile's problem
+            void *out = ti.extra ? p.x_out : p.out;
+            const int64_t ld_out = ti.extra ? p.x_ld_out : p.ld_out;
+            const int n_out = ti.extra ? p.x_n_out : p.n_out;
+            const float *row_scale = ti.extra ? nullptr : p.row_scale;
+            const int64_t rows_cap = ti.extra ? static_cast<int64_t>(p.x_rows) : p.rows_cap;
+            const int64_t split_off = ti.extra ? 0 : ti.ks * p.split_stride;
             if (!ti.swap) {
                 // lane = output row, columns = output features
                 const int64_t row = static_cast<int64_t>(ti.row0) + r_in_tile;
-                const bool row_ok = r_in_tile < ti.rows_valid && row >= 0 && row < p.rows_cap;
+                const bool row_ok = r_in_tile < ti.rows_valid && row >= 0 && row < rows_cap;
                 float scale = 1.0f;
-                if (p.row_scale != nullptr && row_ok)
-                    scale = p.row_scale[row];
+                if (row_scale != nullptr && row_ok)
+                    scale = row_scale[row];
 #pragma unroll 1
                 for (int c = 0; c < OUTN; c += 32) {
                     uint32_t v[32];
@@ -519,8 +578,8 @@ __global__ void __launch_bounds__(kThreads, 1)
                         }
                     }
                     if (row_ok)
-                        store_row32<OUT_F32>(p.out, ti.ks * p.split_stride + row * p.ld_out,
-                                             ti.n0 + c, p.n_out, o);
+                        store_row32<OUT_F32>(out, split_off + row * ld_out,
+                                             ti.n0 + c, n_out, o);
                 }
             } else {
                 // swapped tile: lane = output feature, columns = tokens
@@ -530,8 +589,8 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
                     for (int i = 0; i < 16; ++i) {
                         const int64_t row = static_cast<int64_t>(ti.row0) + c + i;
-                        sc[i] = (p.row_scale != nullptr && c + i < ti.rows_valid && row < p.rows_cap)
-                                    ? p.row_scale[row] : 1.0f;
+                        sc[i] = (row_scale != nullptr && c + i < ti.rows_valid && row < rows_cap)
+                                    ? row_scale[row] : 1.0f;
                     }
                     if (EPI == EPI_SWIGLU) {
                         uint32_t v[16], u[16];
@@ -544,8 +603,8 @@ __global__ void __launch_bounds__(kThreads, 1)
                             const int64_t row = static_cast<int64_t>(ti.row0) + c + i;
                             const float o = silu_f(__uint_as_float(v[i]) * sc[i]) *
                                             (__uint_as_float(u[i]) * sc[i]);
-                            if (c + i < ti.rows_valid && row < p.rows_cap && col < p.n_out)
-                                store_one<OUT_F32>(p.out, ti.ks * p.split_stride + row * p.ld_out + col, o);
+                            if (c + i < ti.rows_valid && row < rows_cap && col < n_out)
+                                store_one<OUT_F32>(out, split_off + row * ld_out + col, o);
                         }
                     } else {
 #pragma unroll
@@ -560,8 +619,8 @@ __global__ void __launch_bounds__(kThreads, 1)
                                 float x = __uint_as_float(v[i]) * sc[i];
                                 if (EPI == EPI_RELU)
                                     x = fmaxf(x, 0.0f);
-                                if (c + i < ti.rows_valid && row < p.rows_cap && col < p.n_out)
-                                    store_one<OUT_F32>(p.out, ti.ks * p.split_stride + row * p.ld_out + col, x);
+                                if (c + i < ti.rows_valid && row < rows_cap && col < n_out)
+                                    store_one<OUT_F32>(out, split_off + row * ld_out + col, x);
                             }
                         }
                     }
@@ -573,7 +632,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         };
         int it = 0;
         for (int t = blockIdx.x; t < total_tiles; t += gridDim.x) {
-            const TileInfo ti = tile_info(t, s_prefix, s_off, G, n_tiles, OUTN, p.ksplit, KB, Geo::REM_ROWS);
+            const TileInfo ti = info(t);
             if (!part(ti, it))
                 break;
             if (ti.combo) {
@@ -682,6 +741,22 @@ cudaError_t launch_impl(const GemmLaunch &L, cudaStream_t stream)
     } else {
         mB2 = mB;
     }
+    // the second problem's maps (copies of the first ones when there is none)
+    CUtensorMap mXA = mA, mXA16 = mA16, mXB = mB, mXB2 = mB2;
+    if (L.x_rows > 0) {
+        if (OUT_F32 || L.ksplit > 1 || !L.XA || !L.XB || !L.x_out)
+            return cudaErrorInvalidValue;
+        if (!make_map_bf16(&mXA, L.XA, L.x_rows, L.XK, BM) ||
+            !make_map_bf16(&mXA16, L.XA, L.x_rows, L.XK, 16) ||
+            !make_map_bf16(&mXB, L.XB, L.x_n_out, L.XK, b_box))
+            return cudaErrorInvalidValue;
+        if (EPI == EPI_SWIGLU) {
+            if (!L.XB2 || !make_map_bf16(&mXB2, L.XB2, L.x_n_out, L.XK, b_box))
+                return cudaErrorInvalidValue;
+        } else {
+            mXB2 = mXB;
+        }
+    }
     static DeviceOnce attr_once;   // per device: function attributes are per device
     cudaError_t e = device_once(attr_once, nullptr, [](int *) {
         return cudaFuncSetAttribute(grouped_gemm_tc<BN, EPI, OUT_F32>,
@@ -700,18 +775,26 @@ cudaError_t launch_impl(const GemmLaunch &L, cudaStream_t stream)
     p.ld_out = L.ld_out;
     p.row_scale = L.row_scale;
     p.rows_cap = L.out_rows;
-    p.prefetch = L.prefetch;
     p.ksplit = L.ksplit > 1 ? L.ksplit : 1;
     p.split_stride = L.split_stride;
     p.status = L.status;
+    p.x_rows = L.x_rows > 0 ? L.x_rows : 0;
+    p.x_K = L.XK;
+    p.x_n_out = L.x_n_out;
+    p.x_out = L.x_out;
+    p.x_ld_out = L.x_ld_out;
+    p.stream_hint = L.stream_hint;
     const int outn = Geo::OUTN;
     const int64_t n_tiles = (L.n_out + outn - 1) / outn;
     const int64_t m_tiles_max = (L.a_rows + BM - 1) / BM + (L.offsets ? L.G : 0);
     int64_t tiles_max = n_tiles * m_tiles_max * p.ksplit;
+    if (p.x_rows > 0)
+        tiles_max += ((p.x_n_out + outn - 1) / outn) * ((p.x_rows + BM - 1) / BM);
     int grid = static_cast<int>(tiles_max < sm_count() ? tiles_max : sm_count());
     if (grid <= 0)
         return cudaSuccess;
-    launch_k(grouped_gemm_tc<BN, EPI, OUT_F32>, grid, kThreads, Geo::SMEM_BYTES, stream, mA, mA16, mB, mB2, p);
+    launch_k(grouped_gemm_tc<BN, EPI, OUT_F32>, grid, kThreads, Geo::SMEM_BYTES, stream, mA, mA16,
+             mB, mB2, mXA, mXA16, mXB, mXB2, p);
     count_launches(1);
     return cudaGetLastError();
 }

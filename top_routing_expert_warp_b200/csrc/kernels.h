@@ -89,10 +89,23 @@ struct GemmLaunch {
     int64_t out_rows;
     int64_t ld_out;
     const float *row_scale;  // [a_rows] or null
-    int32_t prefetch;        // prefetch weight boxes into L2 ahead of their loads
     int32_t ksplit;          // >1: K split into ksplit slices (fp32 partial outputs)
     int64_t split_stride;    // elements between the partial outputs of two slices
     uint32_t *status;
+    // Optional second problem, one-CTA kernel only, bf16 output, no K split:
+    // one group of x_rows rows (0: none) whose tiles are spread through the
+    // grouped problem's tiles (see gemm_tc.cu).
+    const void *XA;          // [x_rows, XK] bf16
+    int32_t x_rows;
+    int32_t XK;
+    const void *XB;          // [x_n_out, XK] bf16
+    const void *XB2;         // SwiGLU's second weight, same shape, or null
+    int32_t x_n_out;
+    void *x_out;             // [x_rows, x_ld_out] bf16
+    int64_t x_ld_out;
+    // One-CTA kernel: weights of groups of at most two m tiles are read once or
+    // twice in a row: load them evict-first from L2 and the rows evict-last.
+    int32_t stream_hint;
 };
 // K slices the router GEMM uses so that its tiles cover the SMs, at most
 // router_ksplit_cap(T, N) (which sizes the workspace's partial-logit buffer).
@@ -121,6 +134,29 @@ cudaError_t launch_simt_gemm_f32(int epi, const float *A, int64_t rows_cap, int3
                                  const float *B, const float *B2, int32_t n_out,
                                  const int32_t *offsets, int32_t G, int32_t w_blocks,
                                  int32_t rows_single, float *out, cudaStream_t stream);
+
+// The whole forward of a small fp32 layer in one launch: see layer_small.cu.
+// Used for fp32 layers without a capacity limit when layer_small_fits().
+struct LayerSmallLaunch {
+    const float *x, *Wg, *bias, *W1, *W3, *W2, *Ws1, *Ws3, *Ws2;   // W3 / Ws*: may be null
+    float *y;
+    int64_t T;
+    int32_t d, N, k, H, Hs;
+    int32_t gate_mode, renormalize, n_groups, topk_groups, swiglu, slot_priority;
+    float alpha;
+    int32_t *topk_idx;
+    float *topk_w;
+    double *p_part;          // [blocks, N] workspace
+    uint32_t *ticket;        // workspace word, 0 between calls
+    int32_t *counts, *offsets, *perm, *inv_row;
+    uint8_t *drop;
+    float *p_mean, *f, *aux_loss;   // may be null
+    uint32_t *status;
+};
+constexpr int64_t kSmallMaxPairs = 8192;
+constexpr size_t kSmallMaxSmem = 96 * 1024;
+bool layer_small_fits(const LayerSmallLaunch &L);
+cudaError_t launch_layer_small(const LayerSmallLaunch &L, cudaStream_t stream);
 
 // Router: see router.cu.
 struct RouterLaunch {

@@ -305,13 +305,34 @@ moe_status run_dispatch(const moe_config &c, const void *x, const int32_t *topk_
     return MOE_OK;
 }
 
+// The always-on shared expert of a layer: every token through one dense FFN.
+struct SharedFfn {
+    const void *x;            // [T, d]
+    int32_t rows;             // T
+    int32_t Hs;
+    const void *W1, *W3, *W2; // Ws1, Ws3 [Hs, d], Ws2 [d, Hs]
+    void *h;                  // [T, Hs]
+    void *y;                  // [T, d]
+};
+
 // Dense FFN over grouped rows: up (with activation) into h, down into out.
 // Group g of the rows uses weight block g % w_blocks (w_blocks = 0: block g).
+// With `shared` (bf16 layers on the one-CTA kernel), the shared expert's
+// tiles run inside the same two launches, and *shared_done is set.
+// Whether the expert FFN of `rows_cap` rows over G groups runs on CTA pairs.
+bool ffn_on_pairs(int64_t rows_cap, int32_t G)
+{
+    return rows_cap >= moe::kPairMinRowsPerGroup * G;
+}
+
 moe_status run_ffn(const moe_config &c, const void *A, const float *row_scale, int64_t rows_cap,
                    const int32_t *offsets, int32_t G, int32_t rows_single, int32_t H,
                    const void *W1, const void *W3, const void *W2, void *h, void *out,
-                   uint32_t *status, cudaStream_t s, int mark_between = -1, int32_t w_blocks = 0)
+                   uint32_t *status, cudaStream_t s, int mark_between = -1, int32_t w_blocks = 0,
+                   const SharedFfn *shared = nullptr, bool *shared_done = nullptr)
 {
+    if (shared_done)
+        *shared_done = false;
     if (rows_cap == 0)
         return MOE_OK;
     const int32_t wb = w_blocks > 0 ? w_blocks : G;
@@ -349,7 +370,24 @@ moe_status run_ffn(const moe_config &c, const void *A, const float *row_scale, i
     U.row_scale = row_scale;
     U.status = status;
     // compute-bound expert projections (many rows per expert) run on CTA pairs
-    const bool pair = rows_cap >= moe::kPairMinRowsPerGroup * G;
+    const bool pair = ffn_on_pairs(rows_cap, G);
+    // groups of at most two 128-row tiles read their weight tiles once or twice
+    // in a row: stream those weights past L2 (evict-first)
+    const int32_t hint = (!pair && offsets != nullptr && rows_cap <= 256 * static_cast<int64_t>(G))
+                             ? 1 : 0;
+    U.stream_hint = hint;
+    // the shared expert's tiles ride in the launches of the routed experts
+    const bool fuse = shared != nullptr && !pair && shared->rows > 0;
+    if (fuse) {
+        U.XA = shared->x;
+        U.x_rows = shared->rows;
+        U.XK = c.d;
+        U.XB = shared->W1;
+        U.XB2 = shared->W3;
+        U.x_n_out = shared->Hs;
+        U.x_out = shared->h;
+        U.x_ld_out = shared->Hs;
+    }
     MOE_CUDA(pair ? moe::launch_grouped_gemm_pair(U, s) : moe::launch_grouped_gemm(U, s));
     if (mark_between >= 0)
         prof_mark(mark_between, s);
@@ -372,7 +410,20 @@ moe_status run_ffn(const moe_config &c, const void *A, const float *row_scale, i
     Dn.ld_out = c.d;
     Dn.row_scale = nullptr;
     Dn.status = status;
+    Dn.stream_hint = hint;
+    if (fuse) {
+        Dn.XA = shared->h;
+        Dn.x_rows = shared->rows;
+        Dn.XK = shared->Hs;
+        Dn.XB = shared->W2;
+        Dn.XB2 = nullptr;
+        Dn.x_n_out = c.d;
+        Dn.x_out = shared->y;
+        Dn.x_ld_out = c.d;
+    }
     MOE_CUDA(pair ? moe::launch_grouped_gemm_pair(Dn, s) : moe::launch_grouped_gemm(Dn, s));
+    if (shared_done)
+        *shared_done = fuse;
     return MOE_OK;
 }
 
@@ -571,6 +622,59 @@ moe_status moe_layer_forward(const moe_config *cfg, const void *x, const void *W
     const bool fp8 = c.dispatch_dtype == MOE_FP8_E4M3;
     int32_t *offsets = w.at<int32_t>(w.L.offsets);
 
+    // small fp32 layers without a capacity limit: the whole forward in one launch
+    if (c.dtype == MOE_F32 && c.capacity_factor <= 0.0f && c.T > 0 &&
+        !(node_limited(c) && c.gate_mode == MOE_GATE_SOFTMAX_THEN_TOPK && !c.renormalize)) {
+        moe::LayerSmallLaunch S{};
+        S.x = static_cast<const float *>(x);
+        S.Wg = static_cast<const float *>(Wg);
+        S.bias = bias;
+        S.W1 = static_cast<const float *>(W1);
+        S.W3 = swiglu ? static_cast<const float *>(W3) : nullptr;
+        S.W2 = static_cast<const float *>(W2);
+        S.Ws1 = shared ? static_cast<const float *>(Ws1) : nullptr;
+        S.Ws3 = (shared && swiglu) ? static_cast<const float *>(Ws3) : nullptr;
+        S.Ws2 = shared ? static_cast<const float *>(Ws2) : nullptr;
+        S.y = static_cast<float *>(y);
+        S.T = c.T;
+        S.d = c.d;
+        S.N = c.N;
+        S.k = c.k;
+        S.H = c.H;
+        S.Hs = c.H_shared;
+        S.gate_mode = c.gate_mode;
+        S.renormalize = c.renormalize;
+        S.n_groups = node_limited(c) ? c.n_groups : 0;
+        S.topk_groups = node_limited(c) ? c.topk_groups : 0;
+        S.swiglu = swiglu ? 1 : 0;
+        S.slot_priority = c.slot_priority;
+        S.alpha = c.aux_alpha;
+        S.topk_idx = idx;
+        S.topk_w = gw;
+        S.p_part = w.at<double>(w.L.p_part);
+        S.ticket = w.status() + 1;
+        S.counts = counts;
+        S.offsets = offsets;
+        S.perm = w.at<int32_t>(w.L.perm);
+        S.inv_row = w.at<int32_t>(w.L.inv_row);
+        S.drop = w.at<uint8_t>(w.L.drop);
+        S.p_mean = pm;
+        S.f = f;
+        S.aux_loss = aux_loss;
+        S.status = w.status();
+        if (moe::layer_small_fits(S)) {
+            // one kernel: its time is reported as the expert stage
+            prof_mark(0, s);
+            prof_mark(1, s);
+            prof_mark(2, s);
+            MOE_CUDA(moe::launch_layer_small(S, s));
+            for (int b = 3; b < kMarks; ++b)
+                prof_mark(b, s);
+            if (g_prof.on && g_prof.steps < g_prof.max_steps)
+                ++g_prof.steps;
+            return MOE_OK;
+        }
+    }
     prof_mark(0, s);
     st = run_router(c, x, Wg, bias, nullptr, idx, gw, pm, w, s);
     if (st != MOE_OK)
@@ -598,16 +702,19 @@ moe_status moe_layer_forward(const moe_config *cfg, const void *x, const void *W
         return MOE_OK;
     }
     const int64_t rows_cap = c.T * c.k;
+    void *ys = shared ? w.at<void>(w.L.ys) : nullptr;
+    SharedFfn sh{x, static_cast<int32_t>(c.T), c.H_shared, Ws1, swiglu ? Ws3 : nullptr, Ws2,
+                 w.at<void>(w.L.hs), ys};
+    bool shared_done = false;
     st = run_ffn(c, xg, fp8 ? w.at<float>(w.L.x_scale) : nullptr, rows_cap, offsets, ffn_groups(c),
                  0, c.H,
                  W1, swiglu ? W3 : nullptr, W2, w.at<void>(w.L.h), w.at<void>(w.L.y_perm),
-                 w.status(), s, 3);
+                 w.status(), s, 3, 0, (shared && c.dtype == MOE_BF16) ? &sh : nullptr,
+                 &shared_done);
     if (st != MOE_OK)
         return st;
     prof_mark(4, s);
-    void *ys = nullptr;
-    if (shared) {
-        ys = w.at<void>(w.L.ys);
+    if (shared && !shared_done) {
         st = run_ffn(c, x, nullptr, c.T, nullptr, 1, static_cast<int32_t>(c.T), c.H_shared, Ws1,
                      swiglu ? Ws3 : nullptr, Ws2, w.at<void>(w.L.hs), ys, w.status(), s);
         if (st != MOE_OK)

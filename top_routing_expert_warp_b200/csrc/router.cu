@@ -24,205 +24,18 @@
 #include "common.cuh"
 #include "kernels.h"
 #include "moe.h"
+#include "router_small.cuh"
 
 namespace moe {
 
 namespace {
 
+using namespace rsel;
+
 constexpr int kThreads = 256;
 constexpr int kWarps = kThreads / 32;
-constexpr int kMaxK = 8;
 constexpr int kMaxCand = 10;
 constexpr int kMaxPerLane = 8;  // large-N path: N <= 256
-
-__device__ __forceinline__ double warp_sum(double v)
-{
-#pragma unroll
-    for (int o = 16; o > 0; o >>= 1)
-        v += __shfl_xor_sync(0xffffffffu, v, o);
-    return v;
-}
-
-// Accumulator of a dot product: a compensated fp32 pair (hi + lo) for bf16
-// operands, whose products are exact in fp32 (8-bit significands); plain fp64
-// for fp32 operands.  Each 16-byte chunk (8 bf16 products) is summed in fp32,
-// then added to (hi, lo) with Knuth's branch-free TwoSum, so no rounding
-// error accumulates across chunks and the result is as accurate as an fp64
-// sum of the chunk sums, without fp64 or conversion instructions in the loop.
-struct DotAcc {
-    float hi = 0.0f, lo = 0.0f;
-    double d = 0.0;
-    __device__ __forceinline__ void add_chunk_sum(float s)
-    {
-        const float t = hi + s;
-        const float bp = t - hi;
-        lo += (hi - (t - bp)) + (s - bp);
-        hi = t;
-    }
-    __device__ __forceinline__ double value(bool bf16) const
-    {
-        return bf16 ? static_cast<double>(hi) + static_cast<double>(lo) : d;
-    }
-};
-
-template <bool BF16>
-__device__ __forceinline__ void chunk_dot(const float (&xf)[8], const uint4 b, DotAcc &acc)
-{
-    const uint32_t bv[4] = {b.x, b.y, b.z, b.w};
-    if (BF16) {
-        float s = xf[0] * __uint_as_float(bv[0] << 16);
-        s = fmaf(xf[1], __uint_as_float(bv[0] & 0xFFFF0000u), s);
-#pragma unroll
-        for (int i = 1; i < 4; ++i) {
-            s = fmaf(xf[2 * i], __uint_as_float(bv[i] << 16), s);
-            s = fmaf(xf[2 * i + 1], __uint_as_float(bv[i] & 0xFFFF0000u), s);
-        }
-        acc.add_chunk_sum(s);
-    } else {
-#pragma unroll
-        for (int i = 0; i < 4; ++i)
-            acc.d = fma(static_cast<double>(xf[i]), static_cast<double>(__uint_as_float(bv[i])),
-                        acc.d);
-    }
-}
-
-// The 8 (bf16) or 4 (fp32) values of a 16-byte chunk as floats.
-template <bool BF16>
-__device__ __forceinline__ void unpack_chunk(const uint4 a, float (&xf)[8])
-{
-    const uint32_t av[4] = {a.x, a.y, a.z, a.w};
-    if (BF16) {
-#pragma unroll
-        for (int i = 0; i < 4; ++i) {
-            xf[2 * i] = __uint_as_float(av[i] << 16);
-            xf[2 * i + 1] = __uint_as_float(av[i] & 0xFFFF0000u);
-        }
-    } else {
-#pragma unroll
-        for (int i = 0; i < 4; ++i) {
-            xf[i] = __uint_as_float(av[i]);
-            xf[4 + i] = 0.0f;
-        }
-    }
-}
-
-// Selection and gates of one token from its N logits (fp64, every lane holds
-// all of them).  Lane e accumulates the softmax probability of expert e into
-// *my_psum.
-template <int NMAX>
-__device__ __forceinline__ void small_select(const double (&acc)[NMAX], int64_t t, int N, int k,
-                                             int gate_mode, int renorm, int n_groups,
-                                             int topk_groups, int lane,
-                                             int32_t *__restrict__ topk_idx,
-                                             float *__restrict__ topk_w, double *my_psum)
-{
-    // node-limited routing: lane g scores node g (sum of its m highest
-    // probabilities, as exp(l - max), largest first), then the topk_groups
-    // best nodes (lower node first on equal scores) are the allowed ones
-    uint32_t allowed = 0xffffffffu;
-    if (n_groups > 1) {
-        const int S = N / n_groups;
-        const int m = (k + topk_groups - 1) / topk_groups;
-        double gmx = acc[0];
-#pragma unroll
-        for (int e = 1; e < NMAX; ++e)
-            if (e < N && acc[e] > gmx)
-                gmx = acc[e];
-        double gs = -1.0;
-        if (lane < n_groups) {
-            gs = 0.0;
-            uint32_t tk = 0;
-#pragma unroll 1
-            for (int r = 0; r < m; ++r) {
-                int bi = -1;
-                double bv = 0.0;
-#pragma unroll
-                for (int e = 0; e < NMAX; ++e) {
-                    if (e < N && e / S == lane && !((tk >> e) & 1u) && (bi < 0 || acc[e] > bv)) {
-                        bi = e;
-                        bv = acc[e];
-                    }
-                }
-                tk |= 1u << bi;
-                gs += exp(bv - gmx);
-            }
-        }
-        uint32_t gtaken = 0;
-#pragma unroll 1
-        for (int j = 0; j < topk_groups; ++j) {
-            double v = (lane < n_groups && !((gtaken >> lane) & 1u)) ? gs : -1.0;
-            int gi = v >= 0.0 ? lane : 32;
-#pragma unroll
-            for (int o = 16; o > 0; o >>= 1) {
-                const double ov = __shfl_xor_sync(0xffffffffu, v, o);
-                const int oi = __shfl_xor_sync(0xffffffffu, gi, o);
-                if (ov > v || (ov == v && oi < gi)) {
-                    v = ov;
-                    gi = oi;
-                }
-            }
-            gtaken |= 1u << gi;
-        }
-        allowed = 0;
-#pragma unroll
-        for (int e = 0; e < NMAX; ++e)
-            if (e < N && ((gtaken >> (e / S)) & 1u))
-                allowed |= 1u << e;
-    }
-    // top-k: strict comparison in ascending expert order -> lowest index wins
-    uint32_t taken = 0;
-    int sel[kMaxK];
-    double val[kMaxK];
-#pragma unroll
-    for (int j = 0; j < kMaxK; ++j) {
-        sel[j] = 0;
-        val[j] = 0.0;
-        if (j < k) {
-            int bi = -1;
-            double bv = 0.0;
-#pragma unroll
-            for (int e = 0; e < NMAX; ++e) {
-                if (e < N && ((allowed >> e) & 1u) && !((taken >> e) & 1u) &&
-                    (bi < 0 || acc[e] > bv)) {
-                    bi = e;
-                    bv = acc[e];
-                }
-            }
-            taken |= 1u << bi;
-            sel[j] = bi;
-            val[j] = bv;
-        }
-    }
-    // full softmax over N, one expert per lane (aux statistic p, mode F gates)
-    const double mx = val[0];
-    double my_l = 0.0;
-#pragma unroll
-    for (int e = 0; e < NMAX; ++e)
-        if (e == lane)
-            my_l = acc[e];
-    const double my_ev = (lane < N) ? exp(my_l - mx) : 0.0;
-    const double Z = warp_sum(my_ev);
-    *my_psum += my_ev / Z;
-    // gates: lane j < k computes slot j
-    double gj = 0.0;
-    int sj = 0;
-#pragma unroll
-    for (int j = 0; j < kMaxK; ++j)
-        if (j == lane) {
-            sj = sel[j];
-            gj = val[j];
-        }
-    if (lane < k)
-        gj = (gate_mode == MOE_GATE_TOPK_THEN_SOFTMAX) ? exp(gj - mx) : exp(gj - mx) / Z;
-    else
-        gj = 0.0;
-    const double gs = warp_sum(gj);
-    const bool norm = (gate_mode == MOE_GATE_TOPK_THEN_SOFTMAX) || renorm;
-    if (lane < k) {
-        topk_idx[t * k + lane] = sj;
-        topk_w[t * k + lane] = static_cast<float>(norm ? gj / gs : gj);
-    }
-}
 
 // Small-N router: a warp takes kTokPerWarp tokens at a time and kUnroll
 // 16-byte chunks per lane per pass, so several loads of x (from HBM) and of
@@ -348,17 +161,30 @@ struct Comp {
     }
 };
 
-__device__ __forceinline__ float chunk_dot8(const float (&xf)[8], const uint4 b)
+// The 8 bf16 values of a 16-byte chunk as 4 packed fp32 pairs (element 2i in
+// the low half, 2i + 1 in the high half of pair i).
+__device__ __forceinline__ void unpack_pairs(const uint4 a, uint64_t (&p)[4])
 {
-    const uint32_t bv[4] = {b.x, b.y, b.z, b.w};
-    float s = xf[0] * __uint_as_float(bv[0] << 16);
-    s = fmaf(xf[1], __uint_as_float(bv[0] & 0xFFFF0000u), s);
+    const uint32_t av[4] = {a.x, a.y, a.z, a.w};
 #pragma unroll
-    for (int i = 1; i < 4; ++i) {
-        s = fmaf(xf[2 * i], __uint_as_float(bv[i] << 16), s);
-        s = fmaf(xf[2 * i + 1], __uint_as_float(bv[i] & 0xFFFF0000u), s);
-    }
-    return s;
+    for (int i = 0; i < 4; ++i)
+        p[i] = static_cast<uint64_t>(av[i] << 16) |
+               (static_cast<uint64_t>(av[i] & 0xFFFF0000u) << 32);
+}
+
+// Sum of the 8 exact bf16 x bf16 products of a chunk with packed fp32 FMAs
+// (two lanes of partial sums: even and odd elements), then the two added.
+__device__ __forceinline__ float chunk_dot8_x2(const uint64_t (&xp)[4], const uint4 b)
+{
+    uint64_t wp[4];
+    unpack_pairs(b, wp);
+    uint64_t acc;
+    asm("mul.rn.f32x2 %0, %1, %2;" : "=l"(acc) : "l"(xp[0]), "l"(wp[0]));
+#pragma unroll
+    for (int i = 1; i < 4; ++i)
+        asm("fma.rn.f32x2 %0, %1, %2, %0;" : "+l"(acc) : "l"(xp[i]), "l"(wp[i]));
+    return __uint_as_float(static_cast<uint32_t>(acc)) +
+           __uint_as_float(static_cast<uint32_t>(acc >> 32));
 }
 
 // Selection from the tensor-core logits (bf16 layers, any N <= 256): one warp
@@ -368,7 +194,15 @@ __device__ __forceinline__ float chunk_dot8(const float (&xf)[8], const uint4 b)
 // candidates are re-ranked on those values (descending, lower index first)
 // and the gates are taken from them.  The full softmax for p (aux loss) uses
 // the recomputed candidates and fp32 exponentials of the other logits.
-constexpr int kSelUnroll = 2;
+// Stages of the per-warp copy ring of the candidate recomputation: deep
+// enough to keep several 512-byte steps of x and every candidate row in
+// flight per warp, within the shared memory of one 8-warp block per SM for
+// the 8- and 10-candidate forms.
+template <int KCM>
+struct Ring {
+    static constexpr int kStages = KCM >= 8 ? 3 : 4;
+    static constexpr int kBytes = kWarps * kStages * (1 + KCM) * 512;
+};
 
 // NPL: logits per lane (N <= 32 NPL); KCM: bound on the candidate count.
 // Both are compile-time so that every loop below has a fixed trip count and
@@ -383,7 +217,10 @@ __global__ void __launch_bounds__(kThreads, NPL >= 8 ? 2 : 3)
                          float *__restrict__ topk_w, double *__restrict__ p_part)
 {
     grid_dep_wait();
-    extern __shared__ double s_pdyn[];  // [kWarps][N]
+    constexpr int kRing = Ring<KCM>::kStages;
+    extern __shared__ __align__(16) uint8_t s_sel[];
+    uint8_t *s_ring = s_sel;                             // [kWarps][kRing][1 + KCM][32 x 16 B]
+    double *s_pdyn = reinterpret_cast<double *>(s_sel);  // [kWarps][N], after the tokens
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int chunks = d / 8;
     // candidates recomputed at fp64-level accuracy: the k selected experts,
@@ -512,28 +349,48 @@ __global__ void __launch_bounds__(kThreads, NPL >= 8 ? 2 : 3)
             }
         }
         // recomputation of the candidates
+        // Each lane streams its own 16-byte chunks (chunk lane + 32 i at step
+        // i) of x and of the KC candidate rows through a ring of kRing stages
+        // in shared memory with cp.async, kRing - 1 steps ahead of the
+        // arithmetic; it reads back only what it copied, so no warp barrier.
         Comp da[KCM];
-        const uint4 *xr = reinterpret_cast<const uint4 *>(x + t * static_cast<int64_t>(d));
-        for (int c0 = lane; c0 < chunks; c0 += 32 * kSelUnroll) {
-            float xf[kSelUnroll][8];
+        {
+            const uint4 *xr = reinterpret_cast<const uint4 *>(x + t * static_cast<int64_t>(d));
+            const int steps = (chunks + 31) / 32;
+            uint8_t *ring = s_ring + static_cast<size_t>(warp) * kRing * (1 + KCM) * 512 + lane * 16;
+            auto issue = [&](int i) {
+                const int ch = lane + 32 * i;
+                const bool live = i < steps && ch < chunks;
+                uint8_t *slot = ring + (i % kRing) * (1 + KCM) * 512;
+                cp_async_16(smem_u32(slot), xr + (live ? ch : 0), live ? 16u : 0u);
 #pragma unroll
-            for (int u = 0; u < kSelUnroll; ++u) {
-                const int ch = c0 + 32 * u;
-                unpack_chunk<true>(ch < chunks ? __ldg(xr + ch) : make_uint4(0, 0, 0, 0), xf[u]);
-            }
+                for (int c = 0; c < KCM; ++c)
+                    if (c < KC)
+                        cp_async_16(smem_u32(slot + (1 + c) * 512),
+                                    reinterpret_cast<const uint4 *>(
+                                        w + static_cast<int64_t>(cand[c]) * d) + (live ? ch : 0),
+                                    live ? 16u : 0u);
+                cp_async_commit();   // one group per step (empty past the end)
+            };
 #pragma unroll
-            for (int c = 0; c < KCM; ++c) {
-                if (c < KC) {
-                    const uint4 *wr =
-                        reinterpret_cast<const uint4 *>(w + static_cast<int64_t>(cand[c]) * d);
+            for (int i = 0; i < kRing - 1; ++i)
+                issue(i);
+            for (int i = 0; i < steps; ++i) {
+                issue(i + kRing - 1);
+                cp_async_wait<kRing - 1>();   // step i's copies of this lane have landed
+                const int ch = lane + 32 * i;
+                if (ch < chunks) {
+                    const uint8_t *slot = ring + (i % kRing) * (1 + KCM) * 512;
+                    uint64_t xp[4];
+                    unpack_pairs(*reinterpret_cast<const uint4 *>(slot), xp);
 #pragma unroll
-                    for (int u = 0; u < kSelUnroll; ++u) {
-                        const int ch = c0 + 32 * u;
-                        if (ch < chunks)
-                            da[c].add(chunk_dot8(xf[u], __ldg(wr + ch)));
-                    }
+                    for (int c = 0; c < KCM; ++c)
+                        if (c < KC)
+                            da[c].add(chunk_dot8_x2(
+                                xp, *reinterpret_cast<const uint4 *>(slot + (1 + c) * 512)));
                 }
             }
+            cp_async_wait_all();
         }
         double acc[KCM];
 #pragma unroll
@@ -628,6 +485,7 @@ __global__ void __launch_bounds__(kThreads, NPL >= 8 ? 2 : 3)
             topk_w[t * k + lane] = static_cast<float>(norm ? gj / gs : gj * zinv);
         }
     }
+    __syncthreads();   // every warp is done with its ring before it holds the sums
 #pragma unroll
     for (int i = 0; i < NPL; ++i) {
         const int e = lane + 32 * i;
@@ -711,23 +569,34 @@ cudaError_t launch_router_small(RouterLaunch &L, cudaStream_t stream)
 }
 
 template <int NPL, int KCM>
-void select_launch(RouterLaunch &L, int grid, size_t smem, cudaStream_t stream)
+cudaError_t select_launch(RouterLaunch &L, int grid, size_t smem_sums, cudaStream_t stream)
 {
-    launch_k(router_select_kernel<NPL, KCM>, grid, kThreads, smem, stream, 
+    const size_t smem = smem_sums > static_cast<size_t>(Ring<KCM>::kBytes)
+                            ? smem_sums : static_cast<size_t>(Ring<KCM>::kBytes);
+    static DeviceOnce attr_once;   // per device: function attributes are per device
+    cudaError_t e = device_once(attr_once, nullptr, [](int *) {
+        return cudaFuncSetAttribute(router_select_kernel<NPL, KCM>,
+                                    cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                    static_cast<int>(227 * 1024));
+    });
+    if (e != cudaSuccess)
+        return e;
+    return launch_k(router_select_kernel<NPL, KCM>, grid, kThreads, smem, stream,
         L.logits_in, L.ksplit, L.logits_out, static_cast<const uint16_t *>(L.x),
         static_cast<const uint16_t *>(L.Wg), L.bias, L.T, L.d, L.N, L.k, L.gate_mode,
         L.renormalize, L.n_groups, L.topk_groups, L.topk_idx, L.topk_w, L.p_part);
 }
 
 template <int NPL>
-void select_launch_kc(RouterLaunch &L, int kc, int grid, size_t smem, cudaStream_t stream)
+cudaError_t select_launch_kc(RouterLaunch &L, int kc, int grid, size_t smem, cudaStream_t stream)
 {
     if (kc <= 2)
-        select_launch<NPL, 2>(L, grid, smem, stream);
-    else if (kc <= 4)
-        select_launch<NPL, 4>(L, grid, smem, stream);
-    else
-        select_launch<NPL, kMaxCand>(L, grid, smem, stream);
+        return select_launch<NPL, 2>(L, grid, smem, stream);
+    if (kc <= 4)
+        return select_launch<NPL, 4>(L, grid, smem, stream);
+    if (kc <= 8)
+        return select_launch<NPL, 8>(L, grid, smem, stream);
+    return select_launch<NPL, kMaxCand>(L, grid, smem, stream);
 }
 
 cudaError_t launch_router_select(RouterLaunch &L, cudaStream_t stream)
@@ -741,16 +610,17 @@ cudaError_t launch_router_select(RouterLaunch &L, cudaStream_t stream)
     int kc = mode_f_raw ? L.k + 2 : L.k;
     if (kc > L.N)
         kc = L.N;
+    cudaError_t e;
     if (L.N <= 32)
-        select_launch_kc<1>(L, kc, grid, smem, stream);
+        e = select_launch_kc<1>(L, kc, grid, smem, stream);
     else if (L.N <= 64)
-        select_launch_kc<2>(L, kc, grid, smem, stream);
+        e = select_launch_kc<2>(L, kc, grid, smem, stream);
     else if (L.N <= 128)
-        select_launch_kc<4>(L, kc, grid, smem, stream);
+        e = select_launch_kc<4>(L, kc, grid, smem, stream);
     else
-        select_launch_kc<kMaxPerLane>(L, kc, grid, smem, stream);
+        e = select_launch_kc<kMaxPerLane>(L, kc, grid, smem, stream);
     count_launches(1);
-    return cudaGetLastError();
+    return e != cudaSuccess ? e : cudaGetLastError();
 }
 
 cudaError_t launch_p_finalize(const double *p_part, int32_t p_blocks, int32_t N, int64_t T,
