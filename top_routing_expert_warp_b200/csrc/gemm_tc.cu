@@ -63,18 +63,6 @@ struct GemmParams {
     int32_t ksplit;          // >1: split K; split s writes its partial sums at out + s*split_stride
     int64_t split_stride;    // elements
     uint32_t *status;
-    // Optional second problem (x_rows > 0): one group of x_rows rows with its
-    // own A (tensor maps tmXA, tmXA16), weights (tmXB, tmXB2), reduction
-    // length x_K and output x_out [x_rows, x_ld_out] (n_out columns = x_n_out),
-    // no row scale and no K split.  Its tiles are spread evenly through the
-    // grouped problem's tiles, so that a compute-bound problem (a layer's
-    // always-on shared expert) runs on the tensor cores while the grouped
-    // problem streams its weights from HBM.
-    int32_t x_rows;
-    int32_t x_K;
-    int32_t x_n_out;
-    void *x_out;
-    int64_t x_ld_out;
     // 1: the grouped problem's weights are streamed once (few rows per group):
     // load the weight tiles of groups of one or two m tiles evict-first from
     // L2, and the rows evict-last, since every n tile of a group reads them
@@ -113,7 +101,6 @@ struct TileInfo {
     int32_t ks, kb0, kb1;   // K split index and its k-block range
     bool combo;             // combined tile: rows_valid = 128 plus rem_rows more
     int32_t rem_rows, rem_ntok;
-    bool extra;             // a tile of the second problem
     int32_t mtiles;         // m tiles of the tile's group
 };
 
@@ -157,47 +144,25 @@ __device__ __forceinline__ TileInfo group_tile(int g, int local, int row_base, i
     ti.ks = ks;
     ti.kb0 = static_cast<int>((static_cast<int64_t>(ks) * KB) / ksplit);
     ti.kb1 = static_cast<int>((static_cast<int64_t>(ks + 1) * KB) / ksplit);
-    ti.extra = false;
     ti.mtiles = mt_g;
     return ti;
 }
 
-// The merged tile list: `routed` tiles of the grouped problem and `extra`
-// tiles of the second problem, the latter at positions t where
-// floor((t + 1) E / total) > floor(t E / total), i.e. evenly spread.
-struct Sched {
-    int routed, extra, total;
-    int x_ntiles, x_KB;
-};
-
-// Locate tile t of the merged list.  Grouped tiles: prefix[g] <= local <
-// prefix[g+1] finds the group.
-__device__ __forceinline__ TileInfo tile_info(int t, const Sched &sc, const int32_t *s_prefix,
+// Locate tile t: prefix[g] <= t < prefix[g+1] finds the group.
+__device__ __forceinline__ TileInfo tile_info(int t, const int32_t *s_prefix,
                                               const int32_t *s_off, int G, int n_tiles,
-                                              int outn, int ksplit, int KB, int rem_max,
-                                              int x_rows)
+                                              int outn, int ksplit, int KB, int rem_max)
 {
-    int local = t;
-    if (sc.extra > 0) {
-        const int c0 = static_cast<int>((static_cast<int64_t>(t) * sc.extra) / sc.total);
-        const int c1 = static_cast<int>((static_cast<int64_t>(t + 1) * sc.extra) / sc.total);
-        if (c1 > c0) {
-            TileInfo ti = group_tile(0, c0, 0, x_rows, sc.x_ntiles, outn, 1, sc.x_KB, rem_max);
-            ti.extra = true;
-            return ti;
-        }
-        local = t - c0;
-    }
-    int lo = 0, hi = G;  // find largest g with prefix[g] <= local
+    int lo = 0, hi = G;  // find largest g with prefix[g] <= t
     while (hi - lo > 1) {
         int mid = (lo + hi) >> 1;
-        if (s_prefix[mid] <= local)
+        if (s_prefix[mid] <= t)
             lo = mid;
         else
             hi = mid;
     }
     const int g = lo;
-    return group_tile(g, local - s_prefix[g], s_off[g], s_off[g + 1] - s_off[g], n_tiles, outn,
+    return group_tile(g, t - s_prefix[g], s_off[g], s_off[g + 1] - s_off[g], n_tiles, outn,
                       ksplit, KB, rem_max);
 }
 
@@ -257,10 +222,7 @@ template <int BN, int EPI, bool OUT_F32>
 __global__ void __launch_bounds__(kThreads, 1)
     grouped_gemm_tc(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmA16,
                     const __grid_constant__ CUtensorMap tmB, const __grid_constant__ CUtensorMap tmB2,
-                    const __grid_constant__ CUtensorMap tmXA,
-                    const __grid_constant__ CUtensorMap tmXA16,
-                    const __grid_constant__ CUtensorMap tmXB,
-                    const __grid_constant__ CUtensorMap tmXB2, GemmParams p)
+                    GemmParams p)
 {
     grid_dep_wait();
     using Geo = Geometry<BN, EPI>;
@@ -307,13 +269,6 @@ __global__ void __launch_bounds__(kThreads, 1)
         tma_prefetch_desc(&tmB);
         if (EPI == EPI_SWIGLU)
             tma_prefetch_desc(&tmB2);
-        if (p.x_rows > 0) {
-            tma_prefetch_desc(&tmXA);
-            tma_prefetch_desc(&tmXA16);
-            tma_prefetch_desc(&tmXB);
-            if (EPI == EPI_SWIGLU)
-                tma_prefetch_desc(&tmXB2);
-        }
     }
     if (warp == 1) {
         tmem_alloc(s_tmem, Geo::TMEM_COLS);
@@ -356,16 +311,9 @@ __global__ void __launch_bounds__(kThreads, 1)
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem_base = *s_tmem;
-    Sched sched;
-    sched.routed = s_prefix[G];
-    sched.x_ntiles = p.x_rows > 0 ? (p.x_n_out + OUTN - 1) / OUTN : 0;
-    sched.extra = p.x_rows > 0 ? m_tiles_of(p.x_rows, Geo::REM_ROWS) * sched.x_ntiles : 0;
-    sched.total = sched.routed + sched.extra;
-    sched.x_KB = (p.x_K + BK - 1) / BK;
-    const int total_tiles = sched.total;
+    const int total_tiles = s_prefix[G];
     auto info = [&](int t) {
-        return tile_info(t, sched, s_prefix, s_off, G, n_tiles, OUTN, p.ksplit, KB, Geo::REM_ROWS,
-                         p.x_rows);
+        return tile_info(t, s_prefix, s_off, G, n_tiles, OUTN, p.ksplit, KB, Geo::REM_ROWS);
     };
 
     if (warp == 0) {
@@ -381,13 +329,10 @@ __global__ void __launch_bounds__(kThreads, 1)
             for (int t = blockIdx.x; t < total_tiles && ok; t += gridDim.x) {
                 const TileInfo ti = info(t);
                 // weights of groups of one or two m tiles are read once or twice in a row
-                const bool hint = p.stream_hint != 0 && !ti.extra && ti.mtiles <= 2;
+                const bool hint = p.stream_hint != 0 && ti.mtiles <= 2;
                 const uint64_t pol_a = hint ? pol_last : 0;
-                const CUtensorMap *mA = ti.extra ? &tmXA : &tmA;
-                const CUtensorMap *mA16 = ti.extra ? &tmXA16 : &tmA16;
-                const CUtensorMap *mB = ti.extra ? &tmXB : &tmB;
-                const CUtensorMap *mB2 = ti.extra ? &tmXB2 : &tmB2;
-                const int brow = ti.extra ? ti.n0 : (ti.g % p.w_blocks) * p.n_out + ti.n0;
+                const CUtensorMap *mA = &tmA, *mA16 = &tmA16, *mB = &tmB, *mB2 = &tmB2;
+                const int brow = (ti.g % p.w_blocks) * p.n_out + ti.n0;
                 const int a_boxes = ti.ntok / 16;          // swapped tile: 16-row boxes
                 const int r_boxes = ti.rem_ntok / 16;      // combined tile: leftover rows
                 const uint32_t bytes =
@@ -542,13 +487,12 @@ __global__ void __launch_bounds__(kThreads, 1)
             }
             tc_fence_after();
             const uint32_t tacc = tmem_base + (static_cast<uint32_t>(q * 32) << 16) + a * BN;
-            // output of the tile's problem
-            void *out = ti.extra ? p.x_out : p.out;
-            const int64_t ld_out = ti.extra ? p.x_ld_out : p.ld_out;
-            const int n_out = ti.extra ? p.x_n_out : p.n_out;
-            const float *row_scale = ti.extra ? nullptr : p.row_scale;
-            const int64_t rows_cap = ti.extra ? static_cast<int64_t>(p.x_rows) : p.rows_cap;
-            const int64_t split_off = ti.extra ? 0 : ti.ks * p.split_stride;
+            void *out = p.out;
+            const int64_t ld_out = p.ld_out;
+            const int n_out = p.n_out;
+            const float *row_scale = p.row_scale;
+            const int64_t rows_cap = p.rows_cap;
+            const int64_t split_off = ti.ks * p.split_stride;
             if (!ti.swap) {
                 // lane = output row, columns = output features
                 const int64_t row = static_cast<int64_t>(ti.row0) + r_in_tile;
@@ -741,22 +685,6 @@ cudaError_t launch_impl(const GemmLaunch &L, cudaStream_t stream)
     } else {
         mB2 = mB;
     }
-    // the second problem's maps (copies of the first ones when there is none)
-    CUtensorMap mXA = mA, mXA16 = mA16, mXB = mB, mXB2 = mB2;
-    if (L.x_rows > 0) {
-        if (OUT_F32 || L.ksplit > 1 || !L.XA || !L.XB || !L.x_out)
-            return cudaErrorInvalidValue;
-        if (!make_map_bf16(&mXA, L.XA, L.x_rows, L.XK, BM) ||
-            !make_map_bf16(&mXA16, L.XA, L.x_rows, L.XK, 16) ||
-            !make_map_bf16(&mXB, L.XB, L.x_n_out, L.XK, b_box))
-            return cudaErrorInvalidValue;
-        if (EPI == EPI_SWIGLU) {
-            if (!L.XB2 || !make_map_bf16(&mXB2, L.XB2, L.x_n_out, L.XK, b_box))
-                return cudaErrorInvalidValue;
-        } else {
-            mXB2 = mXB;
-        }
-    }
     static DeviceOnce attr_once;   // per device: function attributes are per device
     cudaError_t e = device_once(attr_once, nullptr, [](int *) {
         return cudaFuncSetAttribute(grouped_gemm_tc<BN, EPI, OUT_F32>,
@@ -778,23 +706,16 @@ cudaError_t launch_impl(const GemmLaunch &L, cudaStream_t stream)
     p.ksplit = L.ksplit > 1 ? L.ksplit : 1;
     p.split_stride = L.split_stride;
     p.status = L.status;
-    p.x_rows = L.x_rows > 0 ? L.x_rows : 0;
-    p.x_K = L.XK;
-    p.x_n_out = L.x_n_out;
-    p.x_out = L.x_out;
-    p.x_ld_out = L.x_ld_out;
     p.stream_hint = L.stream_hint;
     const int outn = Geo::OUTN;
     const int64_t n_tiles = (L.n_out + outn - 1) / outn;
     const int64_t m_tiles_max = (L.a_rows + BM - 1) / BM + (L.offsets ? L.G : 0);
     int64_t tiles_max = n_tiles * m_tiles_max * p.ksplit;
-    if (p.x_rows > 0)
-        tiles_max += ((p.x_n_out + outn - 1) / outn) * ((p.x_rows + BM - 1) / BM);
     int grid = static_cast<int>(tiles_max < sm_count() ? tiles_max : sm_count());
     if (grid <= 0)
         return cudaSuccess;
     launch_k(grouped_gemm_tc<BN, EPI, OUT_F32>, grid, kThreads, Geo::SMEM_BYTES, stream, mA, mA16,
-             mB, mB2, mXA, mXA16, mXB, mXB2, p);
+             mB, mB2, p);
     count_launches(1);
     return cudaGetLastError();
 }

@@ -400,8 +400,6 @@ bool make_map(CUtensorMap *m, const void *base, int64_t rows, int64_t cols, int 
 template <int EPI>
 cudaError_t launch_pair_impl(const GemmLaunch &L, cudaStream_t stream)
 {
-    if (L.x_rows > 0)
-        return cudaErrorInvalidValue;   // no second problem on CTA pairs
     CUtensorMap mA, mB, mB2;
     if (!make_map(&mA, L.A, L.a_rows, L.K, HBM) || !make_map(&mB, L.B, L.b_rows, L.K, 128))
         return cudaErrorInvalidValue;

@@ -92,17 +92,6 @@ struct GemmLaunch {
     int32_t ksplit;          // >1: K split into ksplit slices (fp32 partial outputs)
     int64_t split_stride;    // elements between the partial outputs of two slices
     uint32_t *status;
-    // Optional second problem, one-CTA kernel only, bf16 output, no K split:
-    // one group of x_rows rows (0: none) whose tiles are spread through the
-    // grouped problem's tiles (see gemm_tc.cu).
-    const void *XA;          // [x_rows, XK] bf16
-    int32_t x_rows;
-    int32_t XK;
-    const void *XB;          // [x_n_out, XK] bf16
-    const void *XB2;         // SwiGLU's second weight, same shape, or null
-    int32_t x_n_out;
-    void *x_out;             // [x_rows, x_ld_out] bf16
-    int64_t x_ld_out;
     // One-CTA kernel: weights of groups of at most two m tiles are read once or
     // twice in a row: load them evict-first from L2 and the rows evict-last.
     int32_t stream_hint;

@@ -305,34 +305,19 @@ moe_status run_dispatch(const moe_config &c, const void *x, const int32_t *topk_
     return MOE_OK;
 }
 
-// The always-on shared expert of a layer: every token through one dense FFN.
-struct SharedFfn {
-    const void *x;            // [T, d]
-    int32_t rows;             // T
-    int32_t Hs;
-    const void *W1, *W3, *W2; // Ws1, Ws3 [Hs, d], Ws2 [d, Hs]
-    void *h;                  // [T, Hs]
-    void *y;                  // [T, d]
-};
-
-// Dense FFN over grouped rows: up (with activation) into h, down into out.
-// Group g of the rows uses weight block g % w_blocks (w_blocks = 0: block g).
-// With `shared` (bf16 layers on the one-CTA kernel), the shared expert's
-// tiles run inside the same two launches, and *shared_done is set.
 // Whether the expert FFN of `rows_cap` rows over G groups runs on CTA pairs.
 bool ffn_on_pairs(int64_t rows_cap, int32_t G)
 {
     return rows_cap >= moe::kPairMinRowsPerGroup * G;
 }
 
+// Dense FFN over grouped rows: up (with activation) into h, down into out.
+// Group g of the rows uses weight block g % w_blocks (w_blocks = 0: block g).
 moe_status run_ffn(const moe_config &c, const void *A, const float *row_scale, int64_t rows_cap,
                    const int32_t *offsets, int32_t G, int32_t rows_single, int32_t H,
                    const void *W1, const void *W3, const void *W2, void *h, void *out,
-                   uint32_t *status, cudaStream_t s, int mark_between = -1, int32_t w_blocks = 0,
-                   const SharedFfn *shared = nullptr, bool *shared_done = nullptr)
+                   uint32_t *status, cudaStream_t s, int mark_between = -1, int32_t w_blocks = 0)
 {
-    if (shared_done)
-        *shared_done = false;
     if (rows_cap == 0)
         return MOE_OK;
     const int32_t wb = w_blocks > 0 ? w_blocks : G;
@@ -376,18 +361,6 @@ moe_status run_ffn(const moe_config &c, const void *A, const float *row_scale, i
     const int32_t hint = (!pair && offsets != nullptr && rows_cap <= 256 * static_cast<int64_t>(G))
                              ? 1 : 0;
     U.stream_hint = hint;
-    // the shared expert's tiles ride in the launches of the routed experts
-    const bool fuse = shared != nullptr && !pair && shared->rows > 0;
-    if (fuse) {
-        U.XA = shared->x;
-        U.x_rows = shared->rows;
-        U.XK = c.d;
-        U.XB = shared->W1;
-        U.XB2 = shared->W3;
-        U.x_n_out = shared->Hs;
-        U.x_out = shared->h;
-        U.x_ld_out = shared->Hs;
-    }
     MOE_CUDA(pair ? moe::launch_grouped_gemm_pair(U, s) : moe::launch_grouped_gemm(U, s));
     if (mark_between >= 0)
         prof_mark(mark_between, s);
@@ -411,19 +384,7 @@ moe_status run_ffn(const moe_config &c, const void *A, const float *row_scale, i
     Dn.row_scale = nullptr;
     Dn.status = status;
     Dn.stream_hint = hint;
-    if (fuse) {
-        Dn.XA = shared->h;
-        Dn.x_rows = shared->rows;
-        Dn.XK = shared->Hs;
-        Dn.XB = shared->W2;
-        Dn.XB2 = nullptr;
-        Dn.x_n_out = c.d;
-        Dn.x_out = shared->y;
-        Dn.x_ld_out = c.d;
-    }
     MOE_CUDA(pair ? moe::launch_grouped_gemm_pair(Dn, s) : moe::launch_grouped_gemm(Dn, s));
-    if (shared_done)
-        *shared_done = fuse;
     return MOE_OK;
 }
 
@@ -702,19 +663,16 @@ moe_status moe_layer_forward(const moe_config *cfg, const void *x, const void *W
         return MOE_OK;
     }
     const int64_t rows_cap = c.T * c.k;
-    void *ys = shared ? w.at<void>(w.L.ys) : nullptr;
-    SharedFfn sh{x, static_cast<int32_t>(c.T), c.H_shared, Ws1, swiglu ? Ws3 : nullptr, Ws2,
-                 w.at<void>(w.L.hs), ys};
-    bool shared_done = false;
     st = run_ffn(c, xg, fp8 ? w.at<float>(w.L.x_scale) : nullptr, rows_cap, offsets, ffn_groups(c),
                  0, c.H,
                  W1, swiglu ? W3 : nullptr, W2, w.at<void>(w.L.h), w.at<void>(w.L.y_perm),
-                 w.status(), s, 3, 0, (shared && c.dtype == MOE_BF16) ? &sh : nullptr,
-                 &shared_done);
+                 w.status(), s, 3);
     if (st != MOE_OK)
         return st;
     prof_mark(4, s);
-    if (shared && !shared_done) {
+    void *ys = nullptr;
+    if (shared) {
+        ys = w.at<void>(w.L.ys);
         st = run_ffn(c, x, nullptr, c.T, nullptr, 1, static_cast<int32_t>(c.T), c.H_shared, Ws1,
                      swiglu ? Ws3 : nullptr, Ws2, w.at<void>(w.L.hs), ys, w.status(), s);
         if (st != MOE_OK)
