@@ -175,14 +175,17 @@ def test_pair_tile_remainders(act):
             assert rel_l2(got[tail:hi], want[tail:hi]) <= 5e-3, (e, "last tile")
 
 
-@pytest.mark.parametrize("act,fp8", [("swiglu", False), ("relu", False), ("swiglu", True)])
-def test_gemm_combined_tiles(act, fp8):
+@pytest.mark.parametrize("act,fp8,d", [("swiglu", False, 256), ("relu", False, 256),
+                                        ("swiglu", True, 256), ("relu", True, 272),
+                                        ("swiglu", True, 264)])
+def test_gemm_combined_tiles(act, fp8, d):
     # one-CTA GEMM (< 512 rows per expert on average): experts a few rows past
     # 128 or 256 (129, 150, 176, 304) put those rows in a combined tile with
     # the last 128; 177 and 200 leave a separate transposed tile, 100 and 20 a
-    # transposed tile alone, 128 a plain one.  FP8: per-row scales in the epilogue.
+    # transposed tile alone, 128 a plain one.  FP8: per-row scales in the
+    # epilogue.  d = 272 and 264 end in a partial K step (zero-filled by TMA).
     counts = np.array([129, 150, 176, 177, 128, 100, 304, 20, 200])
-    wl = synth.Workload("combo", T=int(counts.sum()), d=256, N=len(counts), k=1, H=384, act=act,
+    wl = synth.Workload("combo", T=int(counts.sum()), d=d, N=len(counts), k=1, H=384, act=act,
                         dtype="bf16", gate_mode="R", dispatch="fp8" if fp8 else "", seed=29)
     assert wl.T < 512 * wl.N
     dev, host = upload_inputs(wl)

@@ -23,6 +23,10 @@ SMALL = {
     "mixtral": synth.MIXTRAL.with_(T=300, d=256, H=384),
     "switch": synth.SWITCH.with_(T=1000, d=128, H=256),
     "deepseek": synth.DEEPSEEK.with_(T=200, d=256, H=128, H_shared=128),
+    # FP8 dispatch with a partial last K step in every d-wide GEMM (d = 272
+    # and 264: not multiples of 64; 264 not of 16 either)
+    "deepseek-d272": synth.DEEPSEEK.with_(T=300, d=272, H=192, H_shared=0, seed=31),
+    "deepseek-d264": synth.DEEPSEEK.with_(T=150, d=264, H=128, H_shared=64, seed=32),
     "grok": synth.GROK.with_(d=512, H=1024),
 }
 
