@@ -163,15 +163,20 @@ def up_kernel(wl):
     """(kernel name, source file) of the dominant kernel the library runs for
     this workload: the single-launch kernel for small fp32 layers without a
     capacity limit, else the expert up-projection (fp32 layers: the SIMT
-    kernel; bf16 layers whose experts average at least 512 rows, T k >= 512 N:
-    the CTA-pair kernel; otherwise the one-CTA tensor-core kernel)."""
+    kernel; bf16 layers whose experts average at least 512 rows, T k >= 512 G
+    with G the expert groups, the fallback expert included: the CTA-pair
+    kernel; otherwise the transposed CTA-pair kernel, or with a fallback
+    expert the one-CTA kernel)."""
     if single_launch(wl):
         return "layer_small_f32", "layer_small.cu"
     if wl.dtype == "f32":
         return "grouped_gemm_simt_f32", "ffn_simt.cu"
-    if wl.T * wl.k >= 512 * wl.N:
+    fallback = wl.overflow == "fallback"
+    if wl.T * wl.k >= 512 * (wl.N + (1 if fallback else 0)):
         return "grouped_gemm_tc_pair", "gemm_tc2.cu"
-    return "grouped_gemm_tc", "gemm_tc.cu"
+    if fallback:
+        return "grouped_gemm_tc", "gemm_tc.cu"
+    return "grouped_gemm_tc_pairt", "gemm_tc2t.cu"
 
 
 def traffic_from_profile(kernel_key: str, workload_key: str, source: str):

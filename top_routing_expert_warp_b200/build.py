@@ -19,8 +19,8 @@ INCLUDE = os.path.join(ROOT, "include")
 BUILD = os.path.join(PKG, "_build")
 LIB = os.path.join(PKG, "libmoe_b200.so")
 
-SOURCES = ["moe_abi.cu", "gemm_tc.cu", "router.cu", "dispatch.cu", "combine.cu", "ffn_simt.cu",
-           "dispatch_noalloc.cu", "gemm_tc2.cu", "layer_small.cu"]
+SOURCES = ["moe_abi.cu", "gemm_tc.cu", "gemm_tc2t.cu", "router.cu", "dispatch.cu", "combine.cu",
+           "ffn_simt.cu", "dispatch_noalloc.cu", "gemm_tc2.cu", "layer_small.cu"]
 HEADERS = ["common.cuh", "kernels.h", "router_small.cuh"]
 
 NVCC_FLAGS = ["-gencode", "arch=compute_100a,code=sm_100a", "-O3", "-lineinfo", "-std=c++17",

@@ -117,6 +117,10 @@ cudaError_t launch_grouped_gemm(const GemmLaunch &L, cudaStream_t stream);
 cudaError_t launch_grouped_gemm_pair(const GemmLaunch &L, cudaStream_t stream);
 // Rows per group from which the pair kernel is used.
 constexpr int64_t kPairMinRowsPerGroup = 512;
+// Same contract on CTA pairs with the weights as the MMA's M (tiles of up to
+// 160 rows of one group against 512 weight rows), for the HBM-bound grouped
+// projections below kPairMinRowsPerGroup; needs offsets: see gemm_tc2t.cu.
+cudaError_t launch_grouped_gemm_pairt(const GemmLaunch &L, cudaStream_t stream);
 
 // fp32 CUDA-core grouped GEMM (fp32 layers): see ffn_simt.cu.
 cudaError_t launch_simt_gemm_f32(int epi, const float *A, int64_t rows_cap, int32_t K,

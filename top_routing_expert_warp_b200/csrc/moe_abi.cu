@@ -354,14 +354,23 @@ moe_status run_ffn(const moe_config &c, const void *A, const float *row_scale, i
     U.ld_out = H;
     U.row_scale = row_scale;
     U.status = status;
-    // compute-bound expert projections (many rows per expert) run on CTA pairs
+    // compute-bound expert projections (many rows per expert) run on CTA pairs;
+    // grouped HBM-bound ones on transposed CTA pairs (weights as the MMA's M),
+    // except with a fallback expert: its one group of thousands of rows runs
+    // faster on the one-CTA kernel (m tiles sharing each weight tile through
+    // L2, which the evict-first weights of the small groups leave it)
     const bool pair = ffn_on_pairs(rows_cap, G);
+    const bool pairt = !pair && offsets != nullptr && !has_fallback(c);
+    auto launch = [&](const moe::GemmLaunch &L) {
+        return pair ? moe::launch_grouped_gemm_pair(L, s)
+                    : (pairt ? moe::launch_grouped_gemm_pairt(L, s) : moe::launch_grouped_gemm(L, s));
+    };
     // groups of at most two 128-row tiles read their weight tiles once or twice
     // in a row: stream those weights past L2 (evict-first)
     const int32_t hint = (!pair && offsets != nullptr && rows_cap <= 256 * static_cast<int64_t>(G))
                              ? 1 : 0;
     U.stream_hint = hint;
-    MOE_CUDA(pair ? moe::launch_grouped_gemm_pair(U, s) : moe::launch_grouped_gemm(U, s));
+    MOE_CUDA(launch(U));
     if (mark_between >= 0)
         prof_mark(mark_between, s);
     moe::GemmLaunch Dn{};
@@ -384,7 +393,7 @@ moe_status run_ffn(const moe_config &c, const void *A, const float *row_scale, i
     Dn.row_scale = nullptr;
     Dn.status = status;
     Dn.stream_hint = hint;
-    MOE_CUDA(pair ? moe::launch_grouped_gemm_pair(Dn, s) : moe::launch_grouped_gemm(Dn, s));
+    MOE_CUDA(launch(Dn));
     return MOE_OK;
 }
 
