@@ -111,7 +111,7 @@ class Clocks:
         try:
             self.proc = subprocess.Popen(
                 ["nvidia-smi", "-i", str(self.index), f"--query-gpu={self.FIELDS}",
-                 "--format=csv,noheader,nounits", "-lms", "200"],
+                 "--format=csv,noheader,nounits", "-lms", "50"],
                 stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
         except OSError:
             self.proc = None
@@ -166,7 +166,9 @@ def up_kernel(wl):
     kernel; bf16 layers whose experts average at least 512 rows, T k >= 512 G
     with G the expert groups, the fallback expert included: the CTA-pair
     kernel; otherwise the transposed CTA-pair kernel, or with a fallback
-    expert the one-CTA kernel)."""
+    expert the one-CTA kernel; the up-projection is the dominant kernel, and
+    the down-projection of layers whose experts average more than 64 rows
+    runs on the one-CTA kernel)."""
     if single_launch(wl):
         return "layer_small_f32", "layer_small.cu"
     if wl.dtype == "f32":

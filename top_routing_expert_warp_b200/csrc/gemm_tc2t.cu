@@ -29,11 +29,14 @@
 // Roles as in gemm_tc2.cu: warp 0 lane 0 of each CTA loads that CTA's weight
 // blocks and row half (the second CTA's copies count their bytes on the
 // first CTA's stage barrier); warp 1 allocates TMEM collectively and, in the
-// first CTA, issues the pair MMAs and the multicast commits; warps 2-5 of
+// first CTA, issues the pair MMAs and the multicast commits; warps 2-9 of
 // each CTA drain that CTA's 128 TMEM lanes (its weight rows) for every row
-// of the tile.  No TMA multicast.  Every wait is bounded; on expiry the
-// kernel records a status bit, tells the other roles to stop, waits
-// (bounded) for its copies and MMAs in flight and releases TMEM.
+// of the tile, two warps per lane quarter taking alternate 16-row steps (a
+// tile of 129-160 rows holds both accumulator slots until its epilogue is
+// done, so that epilogue is on the MMAs' path).  No TMA multicast.  Every
+// wait is bounded; on expiry the kernel records a status bit, tells the
+// other roles to stop, waits (bounded) for its copies and MMAs in flight and
+// releases TMEM.
 #include "common.cuh"
 #include "kernels.h"
 
@@ -49,7 +52,8 @@ constexpr int TMAX = 160;                     // rows per tile (both CTAs)
 constexpr int T_BYTES = (TMAX / 2) * BK * 2;  // 10 KB: this CTA's half of the rows
 constexpr int STAGE_BYTES = W_BYTES + T_BYTES;
 constexpr int STAGES = 5;
-constexpr int kThreads = 192;
+constexpr int kEpiWarps = 8;                  // two per TMEM lane quarter
+constexpr int kThreads = 64 + 32 * kEpiWarps;
 constexpr int kMaxGroups = 1024;
 constexpr int TMEM_COLS = 512;
 constexpr int SLOT = 256;                     // columns of one accumulator slot
@@ -167,7 +171,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         for (int a = 0; a < 2; ++a) {
             mbar_init(&acc_full[a], 1);
-            mbar_init(&acc_empty[a], 2 * 4 * 32);   // both CTAs' epilogue threads
+            mbar_init(&acc_empty[a], 2 * kEpiWarps * 32);   // both CTAs' epilogue threads
         }
         mbar_init(drain, 1);
         *s_abort = 0;
@@ -334,8 +338,9 @@ __global__ void __launch_bounds__(kThreads, 1)
             }
         }
     } else {
-        // ================= epilogue (warps 2..5: this CTA's 128 weight rows) =================
+        // ================= epilogue (warps 2..9: this CTA's 128 weight rows) =================
         const int q = warp & 3;   // TMEM lane quarter: weight rows 32q .. 32q+31 of the block
+        const int half = (warp - 2) >> 2;   // the two warps of a quarter take alternate 16-row steps
         const uint32_t leader_acc_empty[2] = {mapa_shared(smem_u32(&acc_empty[0]), 0),
                                               mapa_shared(smem_u32(&acc_empty[1]), 0)};
         const float *row_scale = p.row_scale;
@@ -396,7 +401,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             if (EPI == EPI_SWIGLU) {
                 // a lane's W1 and W3 values of one feature, 16 rows at a time
 #pragma unroll 1
-                for (int c0 = 0; c0 < ti.ntok; c0 += 16) {
+                for (int c0 = 16 * half; c0 < ti.ntok; c0 += 32) {
                     float sc[16], o[16];
                     scales(c0, sc);
                     uint32_t v[16], u[16];
@@ -418,7 +423,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                 for (int j = 0; j < 2; ++j) {
                     const uint32_t tb = j == 0 ? t0 : t1;
 #pragma unroll 1
-                    for (int c0 = 0; c0 < ti.ntok; c0 += 16) {
+                    for (int c0 = 16 * half; c0 < ti.ntok; c0 += 32) {
                         float sc[16], o[16];
                         scales(c0, sc);
                         uint32_t v[16];

@@ -361,16 +361,22 @@ moe_status run_ffn(const moe_config &c, const void *A, const float *row_scale, i
     // L2, which the evict-first weights of the small groups leave it)
     const bool pair = ffn_on_pairs(rows_cap, G);
     const bool pairt = !pair && offsets != nullptr && !has_fallback(c);
-    auto launch = [&](const moe::GemmLaunch &L) {
+    // the down-projection's K is H, often short: with experts of more than 64
+    // rows on average, many transposed tiles hold both TMEM slots (129-160
+    // rows) through their epilogue, which then weighs on tiles of few K steps;
+    // the one-CTA kernel's double buffer was faster there (DeepSeek-shaped
+    // down-projection 1.59 -> 1.53 ms)
+    const bool pairt_down = pairt && rows_cap <= 64 * static_cast<int64_t>(G);
+    auto launch = [&](const moe::GemmLaunch &L, bool t) {
         return pair ? moe::launch_grouped_gemm_pair(L, s)
-                    : (pairt ? moe::launch_grouped_gemm_pairt(L, s) : moe::launch_grouped_gemm(L, s));
+                    : (t ? moe::launch_grouped_gemm_pairt(L, s) : moe::launch_grouped_gemm(L, s));
     };
     // groups of at most two 128-row tiles read their weight tiles once or twice
     // in a row: stream those weights past L2 (evict-first)
     const int32_t hint = (!pair && offsets != nullptr && rows_cap <= 256 * static_cast<int64_t>(G))
                              ? 1 : 0;
     U.stream_hint = hint;
-    MOE_CUDA(launch(U));
+    MOE_CUDA(launch(U, pairt));
     if (mark_between >= 0)
         prof_mark(mark_between, s);
     moe::GemmLaunch Dn{};
@@ -393,7 +399,7 @@ moe_status run_ffn(const moe_config &c, const void *A, const float *row_scale, i
     Dn.row_scale = nullptr;
     Dn.status = status;
     Dn.stream_hint = hint;
-    MOE_CUDA(launch(Dn));
+    MOE_CUDA(launch(Dn, pairt_down));
     return MOE_OK;
 }
 
