@@ -98,26 +98,48 @@ def algorithmic(wl, kept: np.ndarray):
 
 
 class Clocks:
-    """nvidia-smi sampling of SM clocks and throttle reasons during a region."""
-    FIELDS = ("clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.hw_slowdown,"
-              "clocks_event_reasons.hw_thermal_slowdown,clocks_event_reasons.sw_thermal_slowdown,"
-              "clocks_event_reasons.sw_power_cap")
+    """nvidia-smi sampling of SM clocks and throttle reasons.  Started before the
+    warm-up (nvidia-smi takes a moment to start), stopped after the timed
+    region; the summary keeps the samples stamped inside the region (within
+    one sampling period of its ends)."""
+    NAMES = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap",
+             "hw_power_brake_slowdown", "applications_clocks_setting", "sync_boost"]
+
+    BASIC = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
 
     def __init__(self, index: int):
         self.index = index
         self.proc = None
+        self.names = list(self.NAMES)
+        # a driver without one of the extra fields rejects the whole query:
+        # fall back to the four reasons every driver reports
+        try:
+            ok = subprocess.run(["nvidia-smi", "-i", str(index), f"--query-gpu={self.fields()}",
+                                 "--format=csv,noheader"], capture_output=True,
+                                timeout=10).returncode == 0
+        except (OSError, subprocess.TimeoutExpired):
+            ok = False
+        if not ok:
+            self.names = list(self.BASIC)
 
-    def __enter__(self):
+    def fields(self):
+        return ("timestamp,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+                + ",".join("clocks_event_reasons." + n for n in self.names))
+
+    def start(self):
+        import atexit
+        self.out = ""
         try:
             self.proc = subprocess.Popen(
-                ["nvidia-smi", "-i", str(self.index), f"--query-gpu={self.FIELDS}",
+                ["nvidia-smi", "-i", str(self.index), f"--query-gpu={self.fields()}",
                  "--format=csv,noheader,nounits", "-lms", "50"],
                 stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+            atexit.register(self.stop)   # no sampler outlives an error path
         except OSError:
             self.proc = None
         return self
 
-    def __exit__(self, *a):
+    def stop(self):
         self.out = ""
         if self.proc is not None:
             self.proc.terminate()
@@ -126,14 +148,32 @@ class Clocks:
             except subprocess.TimeoutExpired:
                 self.proc.kill()
                 self.out, _ = self.proc.communicate()
+            self.proc = None
 
-    def summary(self):
-        sm, mx, pw, reasons = [], [], [], set()
-        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+    def __enter__(self):
+        return self.start()
+
+    def __exit__(self, *a):
+        self.stop()
+
+    def summary(self, t0=None, t1=None):
+        """Median SM clock and power, max clock, every reason seen active, and the
+        active-reasons bitmasks seen (nvidia-smi's clocks_event_reasons.active), over
+        the samples stamped in [t0 - 0.06 s, t1 + 0.06 s] (host wall clock) when given."""
+        import datetime
+        sm, mx, pw, reasons, masks = [], [], [], set(), set()
         for line in (self.out or "").splitlines():
             f = [x.strip() for x in line.split(",")]
-            if len(f) < 7:
+            if len(f) < 5 + len(self.names):
                 continue
+            if t0 is not None:
+                try:
+                    ts = datetime.datetime.strptime(f[0], "%Y/%m/%d %H:%M:%S.%f").timestamp()
+                except ValueError:
+                    continue
+                if ts < t0 - 0.06 or ts > t1 + 0.06:
+                    continue
+            f = f[1:]
             try:
                 sm.append(float(f[0]))
                 mx.append(float(f[1]))
@@ -143,15 +183,16 @@ class Clocks:
                 pw.append(float(f[2]))
             except ValueError:
                 pass
-            for n, v in zip(names, f[3:7]):
+            masks.add(f[3])
+            for n, v in zip(self.names, f[4:4 + len(self.names)]):
                 if v.lower().startswith("active"):
                     reasons.add(n)
         if not sm:
             return {"sm_mhz": None, "sm_max_mhz": None, "power_w": None, "reasons": [],
-                    "samples": 0}
-        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": max(mx),
+                    "active_masks": [], "samples": 0}
+        return {"sm_mhz": statistics.median(sm), "sm_min_mhz": min(sm), "sm_max_mhz": max(mx),
                 "power_w": statistics.median(pw) if pw else None, "reasons": sorted(reasons),
-                "samples": len(sm)}
+                "active_masks": sorted(masks), "samples": len(sm)}
 
 
 def single_launch(wl) -> bool:
@@ -439,11 +480,13 @@ def measure(wl, dev, args, rank, local, world, dist, headline: bool):
                               dev.get("Ws2"), y if y_out is None else y_out, idx, gw, counts, f, pm,
                               aux, ws, stream)
 
+    clk = Clocks(local).start()   # running (and started up) well before the timed region
     for i in range(args.warmup):
         step(i)
     torch.cuda.synchronize()
     st, word = moe.moe_check_status(ws)
     if st != moe.MOE_OK:
+        clk.stop()
         raise RuntimeError(f"{wl.name}: device status after warm-up: {moe.status_string(st)} "
                            f"({word:#x})")
     C = wl.capacity()
@@ -485,26 +528,29 @@ def measure(wl, dev, args, rank, local, world, dist, headline: bool):
     barrier()
     torch.cuda.synchronize()
     l0 = moe.moe_launch_count()
-    with Clocks(local) as clk:
-        if not flush:
-            e0 = torch.cuda.Event(enable_timing=True)
-            e1 = torch.cuda.Event(enable_timing=True)
-            e0.record(stream)
-            for i in range(args.steps):
-                step(i)
-            e1.record(stream)
-            torch.cuda.synchronize()
-            ms_local = e0.elapsed_time(e1) / args.steps
-        else:
-            evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
-                   for _ in range(args.steps)]
-            for i in range(args.steps):
-                scratch.fill_(i & 0xFF)           # L2 flush, outside the timed events
-                evs[i][0].record(stream)
-                step(i)
-                evs[i][1].record(stream)
-            torch.cuda.synchronize()
-            ms_local = statistics.mean(a.elapsed_time(b) for a, b in evs)
+    t_region = [time.time(), None]
+    if not flush:
+        e0 = torch.cuda.Event(enable_timing=True)
+        e1 = torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        for i in range(args.steps):
+            step(i)
+        e1.record(stream)
+        torch.cuda.synchronize()
+        ms_local = e0.elapsed_time(e1) / args.steps
+    else:
+        evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+               for _ in range(args.steps)]
+        for i in range(args.steps):
+            scratch.fill_(i & 0xFF)           # L2 flush, outside the timed events
+            evs[i][0].record(stream)
+            step(i)
+            evs[i][1].record(stream)
+        torch.cuda.synchronize()
+        ms_local = statistics.mean(a.elapsed_time(b) for a, b in evs)
+    t_region[1] = time.time()
+    clk.stop()
+    clocks = clk.summary(*t_region)
     launches = moe.moe_launch_count() - l0
     barrier()
     ms = max_over_ranks(ms_local, dist, "cuda")
@@ -580,7 +626,7 @@ def measure(wl, dev, args, rank, local, world, dist, headline: bool):
                                     "token batch rotated over 4 resident copies)"),
            "roofline": roof, "layer_roofline": layer,
            "stages_ms": {k: v / max(1, nrec) for k, v in stages.items()},
-           "routing": stats, "clocks": clk.summary(), "config": config_of(wl)}
+           "routing": stats, "clocks": clocks, "config": config_of(wl)}
     if headline:
         rec["e2e"] = e2e
         rec["gpu_launches"] = int(launches)

@@ -218,3 +218,42 @@ def test_gemm_combined_tiles(act, fp8, d):
         tail = lo + (counts[e] // 128) * 128
         if hi > tail and counts[e] > 128:
             assert rel_l2(got[tail:hi], want[tail:hi]) <= tol, (e, "rows past the last 128")
+
+
+@pytest.mark.parametrize("act", ["swiglu", "relu"])
+def test_transposed_tiles_small_experts_with_one_long_group(act):
+    # experts averaging at most 64 rows run both projections on the transposed
+    # CTA-pair kernel: rows are cut into chunks of up to 160 rows (one tile),
+    # a longer group into chunks of at most 128 rows (here 330 -> 3 chunks,
+    # 150 -> one tile of 129-160 rows holding both accumulator slots); empty
+    # experts, single rows and a partial last feature tile (H = 384 and
+    # d = 640 against 256- and 512-feature tiles) around them
+    counts = np.array([330, 1, 0, 17, 150, 0, 32, 0, 3, 0, 0, 64, 0, 0, 0, 2])
+    N = len(counts)
+    wl = synth.Workload("transposed", T=int(counts.sum()), d=640, N=N, k=1, H=384, act=act,
+                        dtype="bf16", gate_mode="R", seed=43)
+    assert wl.T <= 64 * N
+    dev, host = upload_inputs(wl)
+    cfg = cfg_of(wl)
+    ws = moe.workspace(cfg)
+    offsets = np.concatenate([[0], np.cumsum(counts)]).astype(np.int32)
+    yp = torch.zeros((wl.T, wl.d), dtype=torch.bfloat16, device="cuda")
+    moe.moe_expert_ffn(cfg, dev["x"], None, torch.from_numpy(offsets).cuda(), dev["W1"],
+                       dev.get("W3"), dev["W2"], yp, ws)
+    assert moe.moe_check_status(ws)[0] == moe.MOE_OK
+    got = to_f64(yp)
+    xin = oracle.decode(host["x"])
+    exp_of_row = np.repeat(np.arange(N), counts)
+    want = np.empty((wl.T, wl.d))
+    for r in range(wl.T):
+        e = exp_of_row[r]
+        want[r] = oracle.ffn_row(xin[r], host["W1"][e], host["W3"][e] if act == "swiglu" else None,
+                                 host["W2"][e], act)
+    for e in range(N):
+        lo, hi = offsets[e], offsets[e + 1]
+        if hi > lo:
+            assert rel_l2(got[lo:hi], want[lo:hi]) <= 5e-3, e
+            # every row of the long group's chunks, one by one
+            if counts[e] > 128:
+                for r in range(lo, hi, 37):
+                    assert rel_l2(got[r:r + 1], want[r:r + 1]) <= 1e-2, (e, r)
