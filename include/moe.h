@@ -153,6 +153,9 @@ typedef struct moe_workspace_regions {
     size_t inv_row;    /* [T*k] int32, -1 for a dropped pair */
     size_t drop;       /* [T*k] uint8 */
     size_t x_scale;    /* [T*k] fp32 per kept row (FP8 dispatch only) */
+    size_t x_gemm;     /* [T*k, d] the expert-ordered rows the expert GEMMs read, rows < R
+                          meaningful: x's rows (dtype), or for FP8 dispatch the E4M3 codes'
+                          values as bf16 (x_gemm * x_scale per row = the dequantised row) */
     size_t total;      /* = moe_workspace_bytes(cfg) */
 } moe_workspace_regions;
 moe_status moe_workspace_layout(const moe_config *cfg, moe_workspace_regions *out);

@@ -143,12 +143,14 @@ def test_workspace_layout_regions(lib):
                           renormalize=True, dispatch_dtype="fp8")
     r = moe.moe_workspace_layout(cfg)
     assert r["total"] == moe.moe_workspace_bytes(cfg)
-    order = ["topk_idx", "topk_w", "counts", "offsets", "perm", "inv_row", "drop", "x_scale"]
+    order = ["topk_idx", "topk_w", "counts", "offsets", "perm", "inv_row", "drop", "x_scale",
+             "x_gemm"]
     offs = [r[n] for n in order]
     assert all(o % 256 == 0 for o in offs) and offs == sorted(offs) and offs[-1] < r["total"]
     rows = 4096 * 8
     need = {"topk_idx": rows * 4, "topk_w": rows * 4, "counts": 256 * 4, "offsets": 258 * 4,
-            "perm": rows * 4, "inv_row": rows * 4, "drop": rows, "x_scale": rows * 4}
+            "perm": rows * 4, "inv_row": rows * 4, "drop": rows, "x_scale": rows * 4,
+            "x_gemm": rows * 7168 * 2}
     nxt = offs[1:] + [r["total"]]
     for n, o, e in zip(order, offs, nxt):
         assert e - o >= need[n], n

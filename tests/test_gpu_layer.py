@@ -183,3 +183,25 @@ def test_layer_full_size(name):
         _check_layer(wl, run, host, stride, full_check=(wl.T <= 256))
     del run, dev
     torch.cuda.empty_cache()
+
+
+@pytest.mark.parametrize("d", [7168, 8192, 4104])
+def test_fp8_payload_rows_bit_exact(d):
+    # rows of 4097-8192 elements take the quantise-scatter form whose first pass
+    # issues a lane's loads all at once (d = 4104: the last chunks masked); the
+    # layer's expert rows hold, for every kept pair, the E4M3 codes of its token
+    # (as exact bf16 values) and the token's scale, bit for bit
+    wl = synth.DEEPSEEK.with_(T=40, d=d, N=8, k=4, H=64, H_shared=0, seed=50 + d % 7)
+    dev, host = upload_inputs(wl)
+    run = LayerRun(wl, dev)
+    run()
+    assert run.check_status()[0] == moe.MOE_OK
+    R = wl.T * wl.k                       # no capacity: every pair kept
+    perm = moe.workspace_view(run.ws, run.cfg, "perm", torch.int32, R).cpu().numpy()
+    xs = moe.workspace_view(run.ws, run.cfg, "x_scale", torch.float32, R).cpu().numpy()
+    xg = moe.workspace_view(run.ws, run.cfg, "x_gemm", torch.int16, R * d).cpu().numpy()
+    q, sc = oracle.quantize_rows(host["x"][perm // wl.k])
+    assert np.array_equal(xs, sc)
+    vals = oracle.e4m3_table()[q].astype(np.float32)          # exact in bf16
+    want = (vals.view(np.uint32) >> 16).astype(np.uint16)
+    assert np.array_equal(xg.view(np.uint16).reshape(R, d), want)

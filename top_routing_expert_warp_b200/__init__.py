@@ -47,7 +47,8 @@ class moe_config(ctypes.Structure):
 class moe_workspace_regions(ctypes.Structure):
     """Mirror of ``struct moe_workspace_regions`` in include/moe.h."""
     _fields_ = [(n, ctypes.c_size_t) for n in ("topk_idx", "topk_w", "counts", "offsets", "perm",
-                                               "inv_row", "drop", "x_scale", "total")]
+                                               "inv_row", "drop", "x_scale", "x_gemm",
+                                               "total")]
 
 
 class MoeError(RuntimeError):

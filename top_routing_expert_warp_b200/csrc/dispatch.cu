@@ -680,6 +680,74 @@ __global__ void __launch_bounds__(kThreads)
     }
 }
 
+// The same with the token's first pass (the amax) issuing all of a lane's CPL
+// 16-byte loads (chunks lane + 32 i) at once, so the row's reads are in flight
+// together; the second pass finds the row in L1.
+template <int KM, int CPL>
+__global__ void __launch_bounds__(kThreads)
+    quantize_scatter_wide_kernel(const uint8_t *__restrict__ x, int64_t T, int d, int k,
+                                 const int32_t *__restrict__ inv_row, uint8_t *__restrict__ out,
+                                 float *__restrict__ out_scale)
+{
+    grid_dep_wait();
+    const int lane = threadIdx.x & 31;
+    const int64_t nwarps = static_cast<int64_t>(gridDim.x) * kWarps;
+    const int chunks = d / 8;
+    for (int64_t t = static_cast<int64_t>(blockIdx.x) * kWarps + (threadIdx.x >> 5); t < T;
+         t += nwarps) {
+        int32_t rows[KM];
+        const int32_t my_row = lane < k ? inv_row[t * k + lane] : -1;
+#pragma unroll
+        for (int j = 0; j < KM; ++j)
+            rows[j] = __shfl_sync(0xffffffffu, my_row, j);
+        const uint4 *src = reinterpret_cast<const uint4 *>(x + t * static_cast<int64_t>(d) * 2);
+        float amax = 0.0f;
+        {
+            uint4 v[CPL];
+#pragma unroll
+            for (int i = 0; i < CPL; ++i) {
+                const int c = lane + 32 * i;
+                v[i] = c < chunks ? __ldg(src + c) : make_uint4(0, 0, 0, 0);
+            }
+#pragma unroll
+            for (int i = 0; i < CPL; ++i) {
+                const uint32_t w[4] = {v[i].x, v[i].y, v[i].z, v[i].w};
+#pragma unroll
+                for (int q = 0; q < 4; ++q) {
+                    amax = fmaxf(amax, fabsf(__uint_as_float(w[q] << 16)));
+                    amax = fmaxf(amax, fabsf(__uint_as_float(w[q] & 0xFFFF0000u)));
+                }
+            }
+        }
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1)
+            amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, o));
+        const float scale = amax > 0.0f ? __fdiv_rn(amax, 448.0f) : 1.0f;
+        if (lane < k && my_row >= 0)
+            out_scale[my_row] = scale;
+#pragma unroll 1
+        for (int c = lane; c < chunks; c += 32) {
+            const uint4 v = __ldg(src + c);
+            const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+            uint32_t b[4];
+#pragma unroll
+            for (int q = 0; q < 4; ++q) {
+                __nv_fp8_e4m3 lo, hi;
+                lo.__x = __nv_cvt_float_to_fp8(__fdiv_rn(__uint_as_float(w[q] << 16), scale),
+                                               __NV_SATFINITE, __NV_E4M3);
+                hi.__x = __nv_cvt_float_to_fp8(__fdiv_rn(__uint_as_float(w[q] & 0xFFFF0000u), scale),
+                                               __NV_SATFINITE, __NV_E4M3);
+                b[q] = pack_bf16x2(static_cast<float>(lo), static_cast<float>(hi));
+            }
+            const uint4 o = make_uint4(b[0], b[1], b[2], b[3]);
+#pragma unroll
+            for (int j = 0; j < KM; ++j)
+                if (j < k && rows[j] >= 0)
+                    reinterpret_cast<uint4 *>(out + static_cast<int64_t>(rows[j]) * d * 2)[c] = o;
+        }
+    }
+}
+
 int gather_grid(int64_t rows)
 {
     int sms = 148, dev = 0;
@@ -759,7 +827,16 @@ cudaError_t launch_quantize_scatter(const void *x, int64_t T, int32_t d, int32_t
     const uint8_t *xs = static_cast<const uint8_t *>(x);
     uint8_t *o = static_cast<uint8_t *>(out);
     const int grid = gather_grid(T);
-    if (k <= 2)
+    const int cpl = (d / 8 + 31) / 32;   // 16-byte chunks of a row per lane
+    // rows of 4097-8192 elements (the DeepSeek-V3 7168 among them): the first
+    // pass's loads all in flight at once
+    if (k > 2 && cpl > 16 && cpl <= 28)
+        launch_k(quantize_scatter_wide_kernel<8, 28>, grid, kThreads, 0, stream, xs, T, d, k,
+                 inv_row, o, out_scale);
+    else if (k > 2 && cpl > 28 && cpl <= 32)
+        launch_k(quantize_scatter_wide_kernel<8, 32>, grid, kThreads, 0, stream, xs, T, d, k,
+                 inv_row, o, out_scale);
+    else if (k <= 2)
         launch_k(quantize_scatter_kernel<2>, grid, kThreads, 0, stream, xs, T, d, k, inv_row, o,
                  out_scale);
     else

@@ -427,6 +427,7 @@ moe_status moe_workspace_layout(const moe_config *cfg, moe_workspace_regions *ou
     out->inv_row = L.inv_row;
     out->drop = L.drop;
     out->x_scale = L.x_scale;
+    out->x_gemm = L.x_gemm;
     out->total = L.total;
     return MOE_OK;
 }
