@@ -82,3 +82,31 @@ def test_algorithmic_bytes_count_the_fallback_expert():
     assert fb["touched"] == plain["touched"] + 1 and fb["R"] == plain["R"] + 22
     assert fb["bytes"] - plain["bytes"] == 2 * wl.d * wl.H * es     # W1 and W2 (ReLU)
     assert fb["flops"] - plain["flops"] == 22 * 2.0 * 2 * wl.d * wl.H
+
+
+def test_clock_summary_keeps_the_timed_region_and_every_reason():
+    # host-only: samples stamped outside [t0 - 0.06, t1 + 0.06] are dropped, every
+    # reason seen active inside is reported with the raw masks, and the bench's
+    # up_kernel names the kernel each workload's up-projection runs on
+    import datetime
+    import bench
+    import synth
+    c = bench.Clocks.__new__(bench.Clocks)
+    c.names = list(bench.Clocks.NAMES)
+    t0 = 1.0e9
+    def line(t, mhz, mask, active):
+        ts = datetime.datetime.fromtimestamp(t).strftime("%Y/%m/%d %H:%M:%S.%f")[:-3]
+        flags = ["Active" if n in active else "Not Active" for n in c.names]
+        return ", ".join([ts, str(mhz), "1965", "500.0", mask] + flags)
+    c.out = "\n".join([line(t0 - 1.0, 900, "0x8", {"hw_slowdown"}),        # before: dropped
+                       line(t0 + 0.1, 1500, "0x4", {"sw_power_cap"}),
+                       line(t0 + 0.2, 1700, "0x0", set()),
+                       line(t0 + 5.0, 800, "0x40", {"sw_thermal_slowdown"})])  # after: dropped
+    s = c.summary(t0, t0 + 0.3)
+    assert s["samples"] == 2 and s["sm_min_mhz"] == 1500 and s["sm_mhz"] == 1600
+    assert s["reasons"] == ["sw_power_cap"] and s["active_masks"] == ["0x0", "0x4"]
+    assert c.summary()["samples"] == 4
+    assert bench.up_kernel(synth.DEEPSEEK)[0] == "grouped_gemm_tc_pairt"
+    assert bench.up_kernel(synth.MIXTRAL)[0] == "grouped_gemm_tc_pair"
+    assert bench.up_kernel(synth.SWITCH_FALLBACK)[0] == "grouped_gemm_tc"
+    assert bench.up_kernel(synth.TINY_F32)[0] == "layer_small_f32"
